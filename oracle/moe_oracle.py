@@ -1,0 +1,226 @@
+"""Plain fp64 CPU oracle of the routed MoE FFN layer.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or execute this
+module: only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
+(and its ``--impl reference`` arm) use it. It shares no code with the CUDA library; its
+inputs come from the seeded generator in ``synth`` or from the tests themselves.
+
+What it computes, step by step, with the passage each step follows
+(page = "Qwen3.8-Flash-Next" architecture study, section
+"MoE: 512 experts behind a width-640 intermediate", unless stated otherwise):
+
+1. router logits  l[t,e] = sum_h x[t,h] * Wr[e,h] (+ b[e])           -- "Router [T, 512]"
+   (the bias exists only as the synthetic Zipf device of the skewed workload)
+2. top-k selection S(t): the k largest logits, decided on the fp32-rounded logits
+   (the page routes with an FP32 softmax), ties to the lower expert index  -- "Top 10"
+3. p = softmax(l) over all E experts; w_j = p[S_j] / sum_{i in S} p[i]
+   ("Selected router probabilities are normalized")                   -- "+ normalize"
+4. expert(x) = W_down (SiLU(W_gate x) * W_up x), SiLU(z) = z / (1 + exp(-z))
+   (layer formula "expert(x) = ...", hidden_act silu on the 2.4T config page)
+5. shared-expert gate  sigma(w_shared . x), sigma(z) = 1 / (1 + exp(-z))
+6. MoE(x) = sum_{e in S} p_e expert_e(x) + sigma(w_shared x) shared(x)  -- layer formula
+7. dispatch (packing): assignments grouped per expert, token-ascending inside an expert
+   ("Dispatch R tokens", R = 10T, section "Follow the kernels, one layer at a time")
+
+Everything is fp64: bf16 and fp32 inputs convert to fp64 exactly. Matrix products use
+numpy's fp64 matmul as a library primitive; nothing is blocked, fused or reordered
+beyond the definition.
+
+Readings of points the pages leave open (each listed in the design notes):
+* logits are not rounded to bf16 before the softmax; mixing weights stay unrounded;
+* the top-k decision uses fp32-rounded logits with lowest-index tie-break, the gap
+  reported per token is l_(k) - l_(k+1) of the fp64 logits;
+* the shared-expert gate is a length-H bf16 vector without bias;
+* gate|up weights are one [2I][H] tensor per expert, gate rows first.
+
+Parity status: values in general are "parity unpinned by the pages" (no worked numeric
+example of a layer output is printed); the pins are closed forms, special cases, brute
+force on tiny inputs and the pages' shape and parameter counts (tests/test_oracle_pins.py).
+"""
+from __future__ import annotations
+
+from typing import Callable, Optional, Union
+
+import numpy as np
+
+ArrayOrFn = Union[np.ndarray, Callable[[int], np.ndarray]]
+
+
+def bf16_to_f64(u16: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> fp64, exactly (bf16 is the top half of an fp32)."""
+    u = np.asarray(u16, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def silu(z: np.ndarray) -> np.ndarray:
+    """SiLU(z) = z * sigmoid(z) = z / (1 + exp(-z))."""
+    return z / (1.0 + np.exp(-z))
+
+
+def sigmoid(z: np.ndarray) -> np.ndarray:
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+# --------------------------------------------------------------------------- router
+
+def router_logits(x_bf16: np.ndarray, w_router: np.ndarray,
+                  router_bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """l[t,e] = x[t,:] . Wr[e,:] (+ b[e]) in fp64.  x: uint16 [T][H]; Wr: f32 [E][H]."""
+    x = bf16_to_f64(x_bf16)
+    wr = np.asarray(w_router, dtype=np.float32).astype(np.float64)
+    logits = x @ wr.T
+    if router_bias is not None:
+        logits = logits + np.asarray(router_bias, dtype=np.float32).astype(np.float64)[None, :]
+    return logits
+
+
+def topk_select(logits: np.ndarray, k: int):
+    """Top-k expert ids per token and the 10th/11th-style gap.
+
+    Decision on the fp32-rounded logits: larger value first, equal values -> lower
+    expert index first. Returns (ids int32 [T][k] in that order, gap fp64 [T]) where
+    gap = (k-th largest fp64 logit) - ((k+1)-th largest fp64 logit), +inf if k == E.
+    """
+    T, E = logits.shape
+    l32 = logits.astype(np.float32)
+    ids = np.empty((T, k), dtype=np.int32)
+    gap = np.full(T, np.inf)
+    for t in range(T):
+        # lexsort: last key is primary -> sort by (-value, index)
+        order = np.lexsort((np.arange(E), -l32[t].astype(np.float64)))
+        ids[t] = order[:k]
+        if k < E:
+            s = np.sort(logits[t])[::-1]
+            gap[t] = s[k - 1] - s[k]
+    return ids, gap
+
+
+def routing_weights(logits: np.ndarray, ids: np.ndarray) -> np.ndarray:
+    """p = softmax over all E; w[t,j] = p[t,ids[t,j]] / sum_j p[t,ids[t,j]] (fp64)."""
+    m = logits.max(axis=1, keepdims=True)
+    ex = np.exp(logits - m)
+    p = ex / ex.sum(axis=1, keepdims=True)
+    ps = np.take_along_axis(p, ids.astype(np.int64), axis=1)
+    return ps / ps.sum(axis=1, keepdims=True)
+
+
+def shared_gate(x_bf16: np.ndarray, w_shared_gate: np.ndarray) -> np.ndarray:
+    """sigma(w_shared . x[t]) per token, fp64."""
+    return sigmoid(bf16_to_f64(x_bf16) @ bf16_to_f64(w_shared_gate))
+
+
+# --------------------------------------------------------------------------- experts
+
+def swiglu_expert(x64: np.ndarray, w_gate_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
+    """W_down (SiLU(W_gate x) * W_up x) for each row of x64 [n][H].
+
+    w_gate_up: uint16 [2I][H] (rows 0..I-1 gate, I..2I-1 up); w_down: uint16 [H][I].
+    """
+    H = x64.shape[1]
+    two_i, hh = w_gate_up.shape
+    I = two_i // 2
+    assert hh == H and w_down.shape == (H, I), "expert weight shapes"
+    wgu = bf16_to_f64(w_gate_up)
+    g = x64 @ wgu[:I].T
+    u = x64 @ wgu[I:].T
+    h = silu(g) * u
+    return h @ bf16_to_f64(w_down).T
+
+
+def _expert(bank: ArrayOrFn, e: int) -> np.ndarray:
+    return bank(e) if callable(bank) else bank[e]
+
+
+# --------------------------------------------------------------------------- dispatch
+
+def permute(ids: np.ndarray, E: int):
+    """Counting-sort dispatch of the T*k assignments, stable in token order.
+
+    Returns offsets [E+1], sorted_token [R] (token of each packed row), assign_row [T][k]
+    (packed row of assignment (t, j)), sorted_slot [R] (j of each packed row).
+    """
+    T, k = ids.shape
+    counts = np.zeros(E, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            counts[ids[t, j]] += 1
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    fill = offsets[:-1].copy()
+    sorted_token = np.empty(T * k, dtype=np.int64)
+    sorted_slot = np.empty(T * k, dtype=np.int64)
+    assign_row = np.empty((T, k), dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = ids[t, j]
+            p = fill[e]
+            fill[e] += 1
+            sorted_token[p] = t
+            sorted_slot[p] = j
+            assign_row[t, j] = p
+    return offsets, sorted_token, assign_row, sorted_slot
+
+
+# --------------------------------------------------------------------------- layer
+
+def moe_forward(x_bf16: np.ndarray, w_router: np.ndarray, router_bias: Optional[np.ndarray],
+                w_gate_up: ArrayOrFn, w_down: ArrayOrFn, ws_gate_up: np.ndarray,
+                ws_down: np.ndarray, w_shared_gate: np.ndarray, k: int,
+                forced_ids: Optional[np.ndarray] = None) -> dict:
+    """The whole layer for the tokens in x_bf16 (uint16 [T][H]); tokens are independent.
+
+    w_gate_up / w_down: arrays [E][2I][H] / [E][H][I] or callables e -> expert slice.
+    forced_ids: evaluate with these expert ids instead of the top-k (same weights rule).
+    Returns dict(out [T][H] fp64, ids, weights [T][k], gap [T], shared_gate [T],
+    logits [T][E], routed [T][H], shared [T][H]).
+    """
+    x64 = bf16_to_f64(x_bf16)
+    T, H = x64.shape
+    logits = router_logits(x_bf16, w_router, router_bias)
+    ids, gap = topk_select(logits, k)
+    if forced_ids is not None:
+        ids = np.asarray(forced_ids, dtype=np.int32)
+    w = routing_weights(logits, ids)
+    routed = np.zeros((T, H))
+    for e in np.unique(ids):
+        rows, slots = np.nonzero(ids == e)
+        y = swiglu_expert(x64[rows], _expert(w_gate_up, int(e)), _expert(w_down, int(e)))
+        routed[rows] += w[rows, slots][:, None] * y
+    sg = shared_gate(x_bf16, w_shared_gate)
+    shared = swiglu_expert(x64, ws_gate_up, ws_down)
+    out = routed + sg[:, None] * shared
+    return dict(out=out, ids=ids, weights=w, gap=gap, shared_gate=sg, logits=logits,
+                routed=routed, shared=shared)
+
+
+def expert_outputs_packed(x_bf16: np.ndarray, ids: np.ndarray, w_gate_up: ArrayOrFn,
+                          w_down: ArrayOrFn, E: int) -> np.ndarray:
+    """y[p] = expert_{e(p)}(x[sorted_token[p]]) for every packed row p (fp64 [R][H]),
+    in the packed order of ``permute(ids, E)``; the unweighted per-assignment outputs."""
+    x64 = bf16_to_f64(x_bf16)
+    offsets, sorted_token, _, _ = permute(ids, E)
+    y = np.zeros((len(sorted_token), x64.shape[1]))
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if b > a:
+            y[a:b] = swiglu_expert(x64[sorted_token[a:b]], _expert(w_gate_up, e), _expert(w_down, e))
+    return y
+
+
+def combine(y: np.ndarray, y_shared: np.ndarray, assign_row: np.ndarray, weights: np.ndarray,
+            shared_gate_values: np.ndarray) -> np.ndarray:
+    """out[t] = sum_j w[t,j] y[assign_row[t,j]] + sg[t] y_shared[t]  (fp64)."""
+    T, k = assign_row.shape
+    out = np.zeros((T, y.shape[1]))
+    for j in range(k):
+        out += weights[:, j:j + 1].astype(np.float64) * y[assign_row[:, j]].astype(np.float64)
+    out += shared_gate_values[:, None].astype(np.float64) * y_shared.astype(np.float64)
+    return out
+
+
+def forward_inputs(inp, rows=None, forced_ids=None) -> dict:
+    """moe_forward on a ``synth.HostInputs``; ``rows`` selects a token subset."""
+    x = inp.x if rows is None else inp.x[np.asarray(rows)]
+    return moe_forward(x, inp.w_router, inp.router_bias, inp.gate_up, inp.down,
+                       inp.ws_gate_up, inp.ws_down, inp.w_shared_gate, inp.cfg.k,
+                       forced_ids=forced_ids)

@@ -1,0 +1,22 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_libs():
+    """Build the generator libraries once if they are missing (CPU-side, seconds)."""
+    import synth
+
+    if not (os.path.exists(synth.HOST_LIB) and os.path.exists(synth.CUDA_LIB)):
+        synth.build()
+    yield
