@@ -1,0 +1,440 @@
+"""Benchmark of the routed MoE FFN layer on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one whole layer forward (router, top-k, dispatch, grouped SwiGLU GEMMs,
+weighted combine with the gated shared expert) over one batch of T tokens, inputs
+resident in HBM. Default workload: the Flash-Next-shaped decode layer (T=64, hidden 2560,
+512 experts top-10, inter 640, shared 640). Under torchrun each rank runs its own
+replica on its own token batch (weak scaling, no data-path collective); the time is the
+max over ranks of CUDA-event time.
+
+Reported beside the device-timed value:
+* e2e         -- the same metric through moe_layer_forward_host: pinned host x copied in,
+                 layer, out copied back, every step inside the timed region;
+* roofline    -- the dominant kernel's algorithmic bytes per launch / its mean launch
+                 time (CUDA events on the launch stream), against the measured HBM copy
+                 bandwidth in MEASURED_PEAKS.json;
+* cpu_baseline-- the fp64 oracle on the host cores on a bounded token sample (rank 0, N=1);
+* clocks      -- nvidia-smi SM clocks and throttle reasons sampled during the timed region.
+
+--impl reference times the oracle (the only other implementation of this layer) on the
+same workload on the host cores; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s (prefill), µs/layer (decode); % of TC or HBM roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = {  # kernel id -> source file whose hash a stored ncu traffic figure carries
+    "gate_up": ("stream_swiglu.cu", "tc_gemm.cu"),
+    "down": ("stream_swiglu.cu", "tc_gemm.cu"),
+    "router_logits": ("router.cu", "tc_gemm.cu"),
+    "router_topk": ("router.cu",),
+    "permute": ("permute.cu",),
+    "combine": ("combine.cu",),
+}
+# oracle token sample per workload for the CPU baseline (about 10-30 s on a host)
+CPU_SAMPLE = {"tiny": 64, "flash_decode": 16, "flash_prefill": 32, "t24_prefill": 3, "t24_skewed": 3}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampler for one GPU (by UUID)."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str, period_ms: int = 100):
+        self.rows = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                self.rows.append((ts, float(parts[1]), float(parts[2]), parts[5], parts[6], parts[7], parts[8]))
+            except (ValueError, IndexError):
+                continue
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, windows):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "nvidia-smi unavailable"}
+        inside = [r for r in self.rows if any(a - 0.15 <= r[0] <= b + 0.15 for a, b in windows)]
+        note = "samples inside the timed regions"
+        if not inside:
+            inside = self.rows[-5:]
+            note = "timed regions shorter than the sampling period: last samples before stop"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "no samples"}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in inside for i in range(4) if r[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside), "note": note}
+
+
+# --------------------------------------------------------------------------- roofline
+
+def algorithmic_bytes(kernel: str, cfg, n_active: int) -> float:
+    """Bytes a launch of `kernel` must move at least (each operand once)."""
+    T, H, I, Is, R = cfg.T, cfg.H, cfg.I, cfg.Is, cfg.R
+    if kernel == "gate_up":  # activated experts' gate|up + shared gate|up + x + h
+        return (n_active * 2 * I * H + 2 * Is * H + T * H) * 2 + (R * I + T * Is) * 2
+    if kernel == "down":  # activated experts' down + shared down + h in + out (fp32)
+        return (n_active * H * I + H * Is) * 2 + (R * I + T * Is) * 2 + T * H * 4
+    if kernel == "router_logits":
+        return cfg.E * H * 4 + T * H * 2 + T * cfg.E * 4
+    if kernel == "router_topk":
+        return T * cfg.E * 4 + T * H * 2 + T * H * 4
+    if kernel == "permute":
+        return R * 4 * 4
+    if kernel == "combine":
+        return (R + T) * H * 4 + T * H * 4
+    return 0.0
+
+
+def kernel_flops(kernel: str, cfg) -> float:
+    T, H, I, Is, R, E = cfg.T, cfg.H, cfg.I, cfg.Is, cfg.R, cfg.E
+    if kernel == "gate_up":
+        return 4.0 * (R * H * I + T * H * Is)
+    if kernel == "down":
+        return 2.0 * (R * H * I + T * H * Is)
+    if kernel == "router_logits":
+        return 2.0 * T * H * E
+    return 0.0
+
+
+def stored_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_per_launch_bytes\s*=\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256\s*=\s*([0-9a-f]{64})", text)
+    if not m or not h or h.group(1) != source_hash(kernel):
+        return None
+    return float(m.group(1))
+
+
+def source_hash(kernel: str) -> str:
+    hsh = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, ()):
+        p = os.path.join(ROOT, "sparse_moe_expert_fp32_b200", "csrc", f)
+        if os.path.exists(p):
+            hsh.update(open(p, "rb").read())
+    return hsh.hexdigest()
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(cfg, seed: int, ntok: int):
+    """Inputs for timing the oracle on `ntok` sampled tokens (weights made beforehand)."""
+    import numpy as np
+
+    import oracle
+    import synth
+
+    host = synth.host_inputs(cfg, seed=seed)
+    rng = np.random.default_rng(99)
+    rows = sorted(rng.choice(cfg.T, min(ntok, cfg.T), replace=False).tolist())
+    x = host.x[rows]
+    logits = oracle.router_logits(x, host.w_router, host.router_bias)
+    ids, _ = oracle.topk_select(logits, cfg.k)
+    gu = {int(e): host.gate_up(int(e)) for e in np.unique(ids)}
+    dn = {int(e): host.down(int(e)) for e in np.unique(ids)}
+    return host, x, gu, dn, rows
+
+
+def time_oracle(cfg, host, x, gu, dn) -> float:
+    import oracle
+
+    t0 = time.perf_counter()
+    oracle.moe_forward(x, host.w_router, host.router_bias, gu.__getitem__, dn.__getitem__,
+                       host.ws_gate_up, host.ws_down, host.w_shared_gate, cfg.k)
+    return time.perf_counter() - t0
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, seed=0):
+    ntok = CPU_SAMPLE.get(cfg.name, 8)
+    host, x, gu, dn, rows = oracle_sample(cfg, seed, ntok)
+    dt = time_oracle(cfg, host, x, gu, dn)
+    return {"value": len(rows) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} of {cfg.T} tokens of the {cfg.name} layer (seed {seed}), full layer per "
+                      f"token in fp64; expert weights made before timing", "seconds": dt}
+
+
+# --------------------------------------------------------------------------- arms
+
+def dist_setup():
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return None
+    ntok = CPU_SAMPLE.get(cfg.name, 8)
+    host, x, gu, dn, rows = oracle_sample(cfg, 0, ntok)
+    for _ in range(args.warmup):
+        time_oracle(cfg, host, x, gu, dn)
+    total = 0.0
+    for _ in range(args.steps):
+        total += time_oracle(cfg, host, x, gu, dn)
+    value = len(rows) * args.steps / total
+    cores = blas_threads()
+    sample = f"{len(rows)} of {cfg.T} tokens of the {cfg.name} layer per step, fp64 oracle on host cores"
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(cfg, None),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def config_block(cfg, variant):
+    return {"workload": cfg.name, "description": cfg.description, "T": cfg.T, "H": cfg.H, "E": cfg.E,
+            "k": cfg.k, "I": cfg.I, "Is": cfg.Is, "zipf_s": cfg.zipf_s, "zero_rows_pct": cfg.zero_rows_pct,
+            "variant": variant, "accumulate": "fp32", "output": "fp32",
+            "l2": "inputs larger than L2 (expert weight bank exceeds the 126 MB L2)"
+            if cfg.E * 3 * cfg.H * cfg.I * 2 > 126e6 else "L2-resident (tiny layer)",
+            "parallelism": "replicas: one token batch per GPU, no collective"}
+
+
+def run_ours(args, cfg, world, rank, local):
+    import numpy as np
+    import torch
+
+    import sparse_moe_expert_fp32_b200 as moe
+    import synth
+
+    variant = {"auto": moe.MOE_VARIANT_AUTO, "stream": moe.MOE_VARIANT_STREAM,
+               "tc": moe.MOE_VARIANT_TC}[args.variant]
+    moe.moe_set_variant(variant)
+    dev = synth.device_inputs(cfg, seed=0, x_seed=rank, device=f"cuda:{local}")
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s, host_staging=True)
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    w = moe.make_weights(dev)
+
+    moe.moe_layer_forward(s, dev["x"], w, out, ws, topk_ids=ids)
+    st, flags = moe.moe_device_status(ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status {st} ({flags})")
+    n_active = int(np.unique(ids.cpu().numpy()).size)
+    for _ in range(args.warmup):
+        moe.moe_layer_forward(s, dev["x"], w, out, ws)
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(local)
+    uuid = str(getattr(props, "uuid", ""))
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}") if rank == 0 else None
+    if sampler:
+        time.sleep(1.5)  # nvidia-smi start-up
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        import torch.distributed as dist
+
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- device-resident timed region
+    windows = []
+    barrier()
+    torch.cuda.synchronize()
+    moe.moe_profile_enable(True)
+    n0 = moe.moe_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        moe.moe_layer_forward(s, dev["x"], w, out, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    windows.append((w0, time.time()))
+    launches = moe.moe_launch_count() - n0
+    moe.moe_profile_enable(False)
+    prof = moe.moe_profile_collect()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+
+    # ---- end to end through the host-buffer entry point
+    x_host = dev["x"].cpu().pin_memory()
+    out_host = torch.empty((cfg.T, cfg.H), dtype=torch.float32).pin_memory()
+    for _ in range(max(1, min(args.warmup, 3))):
+        moe.moe_layer_forward_host(s, x_host, w, out_host, ws)
+    torch.cuda.synchronize()
+    barrier()
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        moe.moe_layer_forward_host(s, x_host, w, out_host, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    windows.append((w0, time.time()))
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+    if sampler:
+        sampler.stop()
+    st, flags = moe.moe_device_status(ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after timing {st} ({flags})")
+    if rank != 0:
+        return None
+
+    tokens = cfg.T * args.steps * world
+    value = tokens / (ms / 1e3)
+    peaks, peak_kind = load_peaks()
+    kernels = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": None}
+               for k, v in prof.items() if v[1] > 0}
+    tot = sum(v[0] for v in prof.values()) or 1.0
+    for k, v in prof.items():
+        if v[1] > 0:
+            kernels[k]["share"] = v[0] / tot
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
+    bound = "tensor" if kernel_flops(dom, cfg) / max(algorithmic_bytes(dom, cfg, n_active), 1) > 290 else "hbm"
+    per_launch_s = kernels[dom]["ms_per_launch"] / 1e3
+    if bound == "hbm":
+        achieved = algorithmic_bytes(dom, cfg, n_active) / per_launch_s / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved = kernel_flops(dom, cfg) / per_launch_s / 1e12
+        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+                "algorithmic_bytes_per_launch": algorithmic_bytes(dom, cfg, n_active),
+                "activated_experts": n_active,
+                "traffic": stored_traffic(dom, cfg.name)}
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "us_per_layer": 1e3 * ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random router)",
+            "config": config_block(cfg, args.variant), "roofline": roofline,
+            "e2e": {"value": cfg.T * args.steps * world / (ms_e2e / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 4},
+            "gpu_launches": launches, "kernels": kernels,
+            "clocks": sampler.summary(windows) if sampler else None}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    return line
+
+
+def main():
+    import synth
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="flash_decode", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--variant", default="auto", choices=["auto", "stream", "tc"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    cfg = synth.CONFIGS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, cfg, world, rank)
+    else:
+        world, rank, local = dist_setup()
+        line = run_ours(args, cfg, world, rank, local)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+/*
+ * moe.h -- C ABI of the routed Mixture-of-Experts FFN layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (Qwen3.8-Flash-Next architecture study, section "MoE: 512 experts behind a
+ * width-640 intermediate", layer formula and pipeline diagram):
+ *
+ *   expert(x) = W_down (SiLU(W_gate x) * W_up x)
+ *   MoE(x)    = sum_{e in top-k} p_e expert_e(x) + sigmoid(w_shared . x) shared(x)
+ *
+ * computed in the page's five stages "Router [T, 512] -> Top 10 + normalize ->
+ * Dispatch R tokens -> Grouped expert GEMMs -> Weighted combine + gated shared expert".
+ * Each stage is one entry point below; moe_layer_forward runs all of them.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Memory: every pointer argument is DEVICE memory unless its description says HOST.
+ *   The caller allocates and owns every buffer, including the workspace; the library
+ *   never allocates, frees or synchronises on these calls (moe_device_status and the
+ *   profiling calls excepted, which synchronise the given stream).
+ * - Types: "bf16" buffers hold IEEE bfloat16 bit patterns (2 bytes), "fp32" IEEE float.
+ *   Every matrix is dense and row-major with the stated shape; no padding or strides.
+ * - Alignment: every device pointer must be 16-byte aligned (MOE_ERR_INVALID_ARG
+ *   otherwise).
+ * - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Work is enqueued asynchronously; outputs are valid once the stream reaches that point.
+ *   The calls make no host-device synchronisation and can be captured in a CUDA graph.
+ * - Errors: a call returns a moe_status synchronously. Argument errors are reported
+ *   before anything is enqueued. MOE_ERR_CUDA reports a launch error. Errors found by a
+ *   kernel while it runs (an expert id out of range, a bounded wait that ran out) are
+ *   recorded in the workspace's status word and reported by moe_device_status.
+ *   No C++ exception crosses this boundary.
+ * - Empty input: T == 0 is valid and enqueues nothing.
+ * - Shape limits: 1 <= k <= min(E, 32), E <= 1024, H, I, Is multiples of 64,
+ *   T <= 2^20, T*k < 2^31. Other shapes give MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,         /* null/misaligned pointer, bad enum value       */
+  MOE_ERR_UNSUPPORTED = 2,         /* shape outside the limits above                */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < moe_workspace_bytes(shape)         */
+  MOE_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed          */
+  MOE_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device-side wait gave up            */
+  MOE_ERR_DEVICE_BOUNDS = 6        /* a kernel met an expert id outside [0, E)      */
+} moe_status;
+
+/* Layer shape. T tokens, hidden size H, E routed experts, k experts per token,
+ * routed-expert intermediate size I, shared-expert intermediate size Is. */
+typedef struct moe_shape {
+  int32_t T, H, E, k, I, Is;
+} moe_shape;
+
+/* Layer weights (device memory, owned by the caller, read only). */
+typedef struct moe_weights {
+  const float* w_router;    /* fp32 [E][H]   router matrix                                 */
+  const float* router_bias; /* fp32 [E]      added to the logits, or NULL for none         */
+  const void* w_gate_up;    /* bf16 [E][2I][H] per expert: rows 0..I-1 gate, I..2I-1 up   */
+  const void* w_down;       /* bf16 [E][H][I]  per expert down projection                 */
+  const void* ws_gate_up;   /* bf16 [2Is][H]   shared expert gate|up                      */
+  const void* ws_down;      /* bf16 [H][Is]    shared expert down                          */
+  const void* w_shared_gate;/* bf16 [H]        shared-expert output gate vector            */
+} moe_weights;
+
+/* Grouped-GEMM variant used by moe_grouped_swiglu and moe_layer_forward. */
+typedef enum moe_variant {
+  MOE_VARIANT_AUTO = 0,   /* streaming when T*k/E < 16 tokens per expert, else tensor-core */
+  MOE_VARIANT_STREAM = 1, /* weight-streaming CUDA-core kernels (decode-size batches)      */
+  MOE_VARIANT_TC = 2      /* tcgen05/TMEM grouped GEMMs fed by TMA (prefill)               */
+} moe_variant;
+
+/* Kernel ids for the measurement calls below. */
+typedef enum moe_kernel {
+  MOE_K_ROUTER_LOGITS = 0, /* router logits                                   */
+  MOE_K_ROUTER_TOPK = 1,   /* softmax / top-k / renormalise / shared gate     */
+  MOE_K_PERMUTE = 2,       /* the three dispatch kernels, counted together    */
+  MOE_K_GATE_UP = 3,       /* grouped gate|up GEMM with the SwiGLU epilogue    */
+  MOE_K_DOWN = 4,          /* grouped down GEMM (+ fused weighted combine)     */
+  MOE_K_COMBINE = 5,       /* unpermute + weighted combine (staged path)       */
+  MOE_K_OTHER = 6,         /* helpers (router weight split, waits)             */
+  MOE_K_COUNT = 7
+} moe_kernel;
+
+/* Bytes of device workspace the calls below need for `shape` (0 on a bad shape).
+ * One workspace serves all calls; its first bytes hold the device status word.
+ * Calls that share a workspace must not overlap in time on the GPU. */
+size_t moe_workspace_bytes(const moe_shape* shape);
+
+/* Extra bytes moe_layer_forward_host needs on top of moe_workspace_bytes
+ * (device staging for x and out). */
+size_t moe_host_staging_bytes(const moe_shape* shape);
+
+/* Set the status word of a fresh workspace to zero (enqueued on `stream`).
+ * Call once after allocating a workspace; moe_device_status clears it afterwards. */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Stages 1-2: "Router [T, 512]" and "Top 10 + normalize" (MoE section, pipeline
+ * diagram; "Selected router probabilities are normalized"; "Routing uses FP32 softmax").
+ *   logits[t,e] = x[t,:] . w_router[e,:] (+ router_bias[e])    fp32
+ *   topk_ids[t,:] = the k largest logits, larger first, equal logits -> lower index
+ *   topk_w[t,j]   = softmax(logits[t])[id_j] / sum_j softmax(logits[t])[id_j]
+ *   shared_gate[t]= sigmoid(x[t,:] . w_shared_gate)                fp32
+ *   gap[t]        = (k-th largest logit) - ((k+1)-th largest), +inf when k == E
+ * x: bf16 [T][H]. topk_ids: int32 [T][k]; topk_w: fp32 [T][k]; shared_gate: fp32 [T];
+ * gap: fp32 [T] or NULL. Uses weights->w_router, router_bias, w_shared_gate only.
+ */
+moe_status moe_router_topk(const moe_shape* shape, const void* x, const moe_weights* weights,
+                           int32_t* topk_ids, float* topk_w, float* shared_gate, float* gap,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Stage 3: "Dispatch R tokens" (MoE pipeline diagram; R = kT token-expert assignments,
+ * section "Follow the kernels, one layer at a time"). A stable counting sort of the
+ * T*k assignments by expert:
+ *   offsets[e]..offsets[e+1]-1 are the packed rows of expert e   (int32 [E+1])
+ *   sorted_token[p] = token of packed row p, ascending inside an expert (int32 [T*k])
+ *   assign_row[t*k+j] = packed row of assignment (t, j)          (int32 [T*k])
+ * topk_ids: int32 [T][k], each row k distinct ids in [0, E). An id outside [0, E) is
+ * skipped and flagged (MOE_ERR_DEVICE_BOUNDS from moe_device_status); the outputs are
+ * then unspecified. Also records the dispatch in the workspace for the grouped GEMMs.
+ */
+moe_status moe_permute(const moe_shape* shape, const int32_t* topk_ids, int32_t* offsets,
+                       int32_t* sorted_token, int32_t* assign_row, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
+ * Stage 4: "Grouped expert GEMMs" with the layer's expert formula
+ * expert(x) = W_down(SiLU(W_gate x) * W_up x). Unweighted per-assignment outputs:
+ *   y[p,:]        = expert_{e(p)}(x[sorted_token[p],:])   fp32 [T*k][H] (packed order)
+ *   y_shared[t,:] = shared(x[t,:])                         fp32 [T][H]
+ * sorted_token / offsets as produced by moe_permute. The intermediate
+ * h = SiLU(gate) * up is rounded to bf16 before the down projection; accumulation is fp32.
+ */
+moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const int32_t* sorted_token,
+                              const int32_t* offsets, const moe_weights* weights, float* y,
+                              float* y_shared, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Stage 5: "Weighted combine + gated shared expert" (layer formula):
+ *   out[t,:] = sum_{j<k} topk_w[t,j] * y[assign_row[t*k+j],:] + shared_gate[t] * y_shared[t,:]
+ * summed in that order, fp32. out: fp32 [T][H]. Needs no workspace.
+ */
+moe_status moe_unpermute_combine(const moe_shape* shape, const float* y, const float* y_shared,
+                                 const int32_t* assign_row, const float* topk_w,
+                                 const float* shared_gate, float* out, void* stream);
+
+/*
+ * The whole layer, MoE(x) for every token (all five stages). x: bf16 [T][H];
+ * out: fp32 [T][H]. topk_ids / topk_w / gap: optional copies of the routing
+ * (int32 [T][k], fp32 [T][k], fp32 [T]) or NULL. The down GEMM adds its weighted
+ * output and the gated shared expert straight into `out` (fp32 atomic adds), so the
+ * order of the k+1 additions per element is not fixed between runs.
+ */
+moe_status moe_layer_forward(const moe_shape* shape, const void* x, const moe_weights* weights,
+                             float* out, int32_t* topk_ids, float* topk_w, float* gap, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * moe_layer_forward with HOST activations: x_host (bf16 [T][H], HOST memory, pinned
+ * for asynchronous copies) is copied to the device, the layer runs, and out_host
+ * (fp32 [T][H], HOST memory) receives the result; all enqueued on `stream` (the host
+ * buffers must stay valid until the stream reaches that point). The workspace must
+ * hold moe_workspace_bytes + moe_host_staging_bytes.
+ */
+moe_status moe_layer_forward_host(const moe_shape* shape, const void* x_host,
+                                  const moe_weights* weights, float* out_host, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* Choose the grouped-GEMM variant for later calls (process-wide; default AUTO). */
+moe_status moe_set_variant(moe_variant variant);
+
+/* Synchronise `stream`, read the workspace status word (MOE_OK, MOE_ERR_DEVICE_BOUNDS
+ * or MOE_ERR_DEVICE_TIMEOUT), and clear it. `detail` (HOST, may be NULL) receives
+ * the raw flag bits. */
+moe_status moe_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* detail);
+
+/* Failure-detection check: enqueue a kernel that waits for *flag != 0 (device int32)
+ * for at most timeout_ns nanoseconds (capped at 10 s), then records MOE_ERR_DEVICE_TIMEOUT in the
+ * workspace status word and returns. The wait is the same bounded wait the pipelined
+ * kernels use. Never hangs. */
+moe_status moe_debug_wait_flag(const int32_t* flag, uint64_t timeout_ns, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* Measurement: while enabled, every kernel launch records a CUDA event pair on its
+ * stream. moe_profile_collect synchronises those events and returns, per moe_kernel
+ * id, the summed device time in ms (HOST float[MOE_K_COUNT]) and the launch counts
+ * (HOST int32[MOE_K_COUNT]), then forgets them. At most 65536 launches are recorded. */
+moe_status moe_profile_enable(int32_t on);
+moe_status moe_profile_collect(float* total_ms, int32_t* launches);
+
+/* Number of kernels this library has launched since it was loaded. */
+uint64_t moe_launch_count(void);
+
+/* Short text for a status code (static storage). */
+const char* moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

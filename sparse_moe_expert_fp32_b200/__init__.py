@@ -1,0 +1,248 @@
+"""Routed MoE FFN layer for NVIDIA B200 (sm_100a): Python binding of ``include/moe.h``.
+
+The layer (Qwen3.8-Flash-Next architecture study, MoE section):
+
+    expert(x) = W_down (SiLU(W_gate x) * W_up x)
+    MoE(x)    = sum_{e in top-k} p_e expert_e(x) + sigmoid(w_shared . x) shared(x)
+
+Every step runs in the CUDA kernels of ``libmoe_b200.so``; this module only marshals
+arguments (torch tensors -> device pointers, the current torch stream) and turns status
+codes into exceptions. There is no CPU path: if the library is missing, importing this
+package raises.
+
+Names follow the C ABI: moe_router_topk, moe_permute, moe_grouped_swiglu,
+moe_unpermute_combine, moe_layer_forward, moe_layer_forward_host, ...
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_WORKSPACE_TOO_SMALL = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_DEVICE_TIMEOUT = 5
+MOE_ERR_DEVICE_BOUNDS = 6
+
+MOE_VARIANT_AUTO = 0
+MOE_VARIANT_STREAM = 1
+MOE_VARIANT_TC = 2
+
+KERNELS = ("router_logits", "router_topk", "permute", "gate_up", "down", "combine", "other")
+MOE_K_COUNT = len(KERNELS)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("T", "H", "E", "k", "I", "Is")]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "router_bias", "w_gate_up", "w_down",
+                                               "ws_gate_up", "ws_down", "w_shared_gate")]
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python sparse_moe_expert_fp32_b200/build.py` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _sz, _i32, _u64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_uint64
+_SP = ctypes.POINTER(moe_shape)
+_WP = ctypes.POINTER(moe_weights)
+
+_SIGS = {
+    "moe_workspace_bytes": ([_SP], _sz),
+    "moe_host_staging_bytes": ([_SP], _sz),
+    "moe_workspace_init": ([_vp, _sz, _vp], ctypes.c_int),
+    "moe_router_topk": ([_SP, _vp, _WP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_permute": ([_SP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_grouped_swiglu": ([_SP, _vp, _vp, _vp, _WP, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_unpermute_combine": ([_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moe_layer_forward": ([_SP, _vp, _WP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_layer_forward_host": ([_SP, _vp, _WP, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_set_variant": ([ctypes.c_int], ctypes.c_int),
+    "moe_device_status": ([_vp, _sz, _vp, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+    "moe_debug_wait_flag": ([_vp, _u64, _vp, _sz, _vp], ctypes.c_int),
+    "moe_profile_enable": ([_i32], ctypes.c_int),
+    "moe_profile_collect": ([ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32)],
+                            ctypes.c_int),
+    "moe_launch_count": ([], _u64),
+    "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.moe_status_string(int(status)).decode()
+
+
+moe_status_string = status_string
+
+
+def _check(status: int, where: str) -> None:
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+# --------------------------------------------------------------------------- marshalling
+
+def _ptr(t) -> Optional[int]:
+    """Device (or host) address of a torch tensor, None for None, ints pass through."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_shape(T: int, H: int, E: int, k: int, I: int, Is: int) -> moe_shape:
+    return moe_shape(T, H, E, k, I, Is)
+
+
+def shape_of(cfg, T: Optional[int] = None) -> moe_shape:
+    """moe_shape of a layer config object with fields T, H, E, k, I, Is."""
+    return moe_shape(cfg.T if T is None else T, cfg.H, cfg.E, cfg.k, cfg.I, cfg.Is)
+
+
+def make_weights(w: dict) -> moe_weights:
+    """moe_weights from a dict of device tensors keyed like the C struct."""
+    return moe_weights(_ptr(w["w_router"]), _ptr(w.get("router_bias")), _ptr(w["w_gate_up"]),
+                       _ptr(w["w_down"]), _ptr(w["ws_gate_up"]), _ptr(w["ws_down"]),
+                       _ptr(w["w_shared_gate"]))
+
+
+def _w(weights) -> moe_weights:
+    return weights if isinstance(weights, moe_weights) else make_weights(weights)
+
+
+def _nbytes(ws) -> int:
+    return ws.numel() * ws.element_size()
+
+
+# --------------------------------------------------------------------------- entry points
+
+def moe_workspace_bytes(shape: moe_shape) -> int:
+    n = _lib.moe_workspace_bytes(ctypes.byref(shape))
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_workspace_bytes")
+    return n
+
+
+def moe_host_staging_bytes(shape: moe_shape) -> int:
+    return _lib.moe_host_staging_bytes(ctypes.byref(shape))
+
+
+def moe_workspace_init(ws, stream=None) -> None:
+    _check(_lib.moe_workspace_init(_ptr(ws), _nbytes(ws), _stream(stream)), "moe_workspace_init")
+
+
+def moe_router_topk(shape, x, weights, topk_ids, topk_w, shared_gate, gap, ws, stream=None):
+    w = _w(weights)
+    _check(_lib.moe_router_topk(ctypes.byref(shape), _ptr(x), ctypes.byref(w), _ptr(topk_ids),
+                                _ptr(topk_w), _ptr(shared_gate), _ptr(gap), _ptr(ws), _nbytes(ws),
+                                _stream(stream)), "moe_router_topk")
+
+
+def moe_permute(shape, topk_ids, offsets, sorted_token, assign_row, ws, stream=None):
+    _check(_lib.moe_permute(ctypes.byref(shape), _ptr(topk_ids), _ptr(offsets), _ptr(sorted_token),
+                            _ptr(assign_row), _ptr(ws), _nbytes(ws), _stream(stream)), "moe_permute")
+
+
+def moe_grouped_swiglu(shape, x, sorted_token, offsets, weights, y, y_shared, ws, stream=None):
+    w = _w(weights)
+    _check(_lib.moe_grouped_swiglu(ctypes.byref(shape), _ptr(x), _ptr(sorted_token), _ptr(offsets),
+                                   ctypes.byref(w), _ptr(y), _ptr(y_shared), _ptr(ws), _nbytes(ws),
+                                   _stream(stream)), "moe_grouped_swiglu")
+
+
+def moe_unpermute_combine(shape, y, y_shared, assign_row, topk_w, shared_gate, out, stream=None):
+    _check(_lib.moe_unpermute_combine(ctypes.byref(shape), _ptr(y), _ptr(y_shared), _ptr(assign_row),
+                                      _ptr(topk_w), _ptr(shared_gate), _ptr(out), _stream(stream)),
+           "moe_unpermute_combine")
+
+
+def moe_layer_forward(shape, x, weights, out, ws, topk_ids=None, topk_w=None, gap=None, stream=None):
+    w = _w(weights)
+    _check(_lib.moe_layer_forward(ctypes.byref(shape), _ptr(x), ctypes.byref(w), _ptr(out),
+                                  _ptr(topk_ids), _ptr(topk_w), _ptr(gap), _ptr(ws), _nbytes(ws),
+                                  _stream(stream)), "moe_layer_forward")
+
+
+def moe_layer_forward_host(shape, x_host, weights, out_host, ws, stream=None):
+    w = _w(weights)
+    _check(_lib.moe_layer_forward_host(ctypes.byref(shape), _ptr(x_host), ctypes.byref(w),
+                                       _ptr(out_host), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "moe_layer_forward_host")
+
+
+def moe_set_variant(variant: int) -> None:
+    _check(_lib.moe_set_variant(int(variant)), "moe_set_variant")
+
+
+def moe_device_status(ws, stream=None):
+    """Returns (status, flag bits); the status word is cleared."""
+    d = ctypes.c_uint32(0)
+    st = _lib.moe_device_status(_ptr(ws), _nbytes(ws), _stream(stream), ctypes.byref(d))
+    return st, d.value
+
+
+def moe_debug_wait_flag(flag, timeout_ns: int, ws, stream=None) -> None:
+    _check(_lib.moe_debug_wait_flag(_ptr(flag), int(timeout_ns), _ptr(ws), _nbytes(ws),
+                                    _stream(stream)), "moe_debug_wait_flag")
+
+
+def moe_profile_enable(on: bool) -> None:
+    _check(_lib.moe_profile_enable(1 if on else 0), "moe_profile_enable")
+
+
+def moe_profile_collect() -> dict:
+    """{kernel name: (total ms, launches)} for the launches recorded since enabling."""
+    ms = (ctypes.c_float * MOE_K_COUNT)()
+    n = (ctypes.c_int32 * MOE_K_COUNT)()
+    _check(_lib.moe_profile_collect(ms, n), "moe_profile_collect")
+    return {KERNELS[i]: (float(ms[i]), int(n[i])) for i in range(MOE_K_COUNT)}
+
+
+def moe_launch_count() -> int:
+    return int(_lib.moe_launch_count())
+
+
+# --------------------------------------------------------------------------- conveniences
+
+def alloc_workspace(shape: moe_shape, device="cuda", host_staging: bool = False, stream=None):
+    """A uint8 device tensor sized for `shape`, with its status word cleared."""
+    import torch
+
+    n = moe_workspace_bytes(shape) + (moe_host_staging_bytes(shape) if host_staging else 0)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    moe_workspace_init(ws, stream)
+    return ws

@@ -1,0 +1,112 @@
+// moe_internal.h -- workspace layout, dispatch plan and launch declarations shared by the
+// translation units of libmoe_b200.so. Not part of the public ABI (include/moe.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kMaxE = 1024;
+constexpr int kMaxK = 32;
+constexpr int kPermBlock = 256;  // tokens per dispatch block (one bit per token in a mask)
+constexpr int kTcChunk = 256;    // max tokens (MMA N) per tensor-core tile
+constexpr uint32_t kFlagBounds = 1u;
+constexpr uint32_t kFlagTimeout = 2u;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Byte offsets of the workspace regions (all 256-byte aligned).
+struct Layout {
+  size_t status;        // uint32 [64]: [0] = error flags, [1..] = diagnostics
+  size_t logits;        // fp32 [T][E]
+  size_t wr_split;      // bf16 [E][3H]: router matrix as hi|mid|lo bf16 pieces (tensor-core router)
+  size_t ids;           // int32 [T][k]
+  size_t w;             // fp32 [T][k]
+  size_t sgate;         // fp32 [T]
+  size_t gap;           // fp32 [T]
+  size_t blk_mask;      // uint32 [nblk][E][8]: token bitmask per dispatch block and expert
+  size_t blk_base;      // int32 [nblk][E]: first packed row of (block, expert)
+  size_t offsets;       // int32 [E+2]
+  size_t sorted_token;  // int32 [T*k]
+  size_t sorted_w;      // fp32 [T*k]: routing weight of each packed row
+  size_t assign_row;    // int32 [T*k]
+  size_t plan;          // int32 plan arrays (see PlanView)
+  size_t h;             // bf16 [T*k + T][ldh]: SwiGLU intermediate, routed rows then shared rows
+  size_t total;
+  int nblk;
+  int ldh;              // max(I, Is)
+};
+
+Layout layout(const moe_shape& s);
+
+// Dispatch plan: groups 0..E-1 are the routed experts, group E the shared expert
+// (all T tokens in order). Group g owns packed rows [row0[g], row0[g+1]) of h.
+struct PlanView {
+  int* n_active;  // [1]
+  int* active;    // [E+1] group ids with >= 1 row, ascending
+  int* row0;      // [E+2]
+  int* tp1;       // [E+2] tile prefix of the tensor-core gate|up GEMM
+  int* tp2;       // [E+2] tile prefix of the tensor-core down GEMM
+};
+
+__host__ __device__ inline size_t plan_ints(int E) { return 1 + (size_t)(E + 1) + 3 * (size_t)(E + 2); }
+
+__host__ __device__ inline PlanView plan_view(void* base, int E) {
+  int* p = static_cast<int*>(base);
+  PlanView v;
+  v.n_active = p;
+  v.active = p + 1;
+  v.row0 = v.active + (E + 1);
+  v.tp1 = v.row0 + (E + 2);
+  v.tp2 = v.tp1 + (E + 2);
+  return v;
+}
+
+// Tensor-core tiling of group g with n rows: ceil(n/256) token chunks, split evenly
+// into chunks that are multiples of 16 rows.
+__host__ __device__ inline int tc_nchunks(int n) { return (n + kTcChunk - 1) / kTcChunk; }
+
+// ---------------------------------------------------------------- launch bookkeeping
+
+// RAII: counts a launch and, while profiling is on, brackets it with CUDA events.
+struct LaunchScope {
+  LaunchScope(moe_kernel id, cudaStream_t s, int nkernels = 1);
+  ~LaunchScope();
+  int slot;
+  cudaStream_t stream;
+};
+
+// ---------------------------------------------------------------- kernel launches
+// Every launcher enqueues on `st` and returns cudaGetLastError().
+
+cudaError_t launch_router_logits_stream(const moe_shape& s, const uint16_t* x, const float* wr,
+                                        float* logits, cudaStream_t st);
+// router logits by the best available kernel for the shape (uses the workspace)
+cudaError_t launch_router_logits(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
+                                 const float* wr, float* logits, cudaStream_t st);
+cudaError_t launch_router_topk(const moe_shape& s, const float* logits, const float* bias,
+                               const uint16_t* x, const uint16_t* wsg, int32_t* ids, float* w,
+                               float* sgate, float* gap, float* out_zero, cudaStream_t st);
+cudaError_t launch_permute(const moe_shape& s, const Layout& L, char* ws, const int32_t* ids,
+                           const float* topk_w, int32_t* offsets, int32_t* sorted_token,
+                           float* sorted_w, int32_t* assign_row, cudaStream_t st);
+cudaError_t launch_plan_from_offsets(const moe_shape& s, const Layout& L, char* ws,
+                                     const int32_t* offsets, cudaStream_t st);
+cudaError_t launch_stream_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
+                                  const int32_t* sorted_token, const moe_weights& w,
+                                  cudaStream_t st);
+cudaError_t launch_stream_down(const moe_shape& s, const Layout& L, char* ws,
+                               const int32_t* sorted_token, const float* sorted_w,
+                               const float* sgate, const moe_weights& w, float* y,
+                               float* y_shared, float* out, cudaStream_t st);
+cudaError_t launch_combine(const moe_shape& s, const float* y, const float* y_shared,
+                           const int32_t* assign_row, const float* topk_w, const float* sgate,
+                           float* out, cudaStream_t st);
+cudaError_t launch_wait_flag(const int32_t* flag, uint64_t timeout_ns, uint32_t* status,
+                             cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,240 @@
+// permute.cu -- stage 3 of the layer, "Dispatch R tokens" (Qwen3.8-Flash-Next
+// architecture study, MoE pipeline diagram; R = kT token-expert assignments, section
+// "Follow the kernels, one layer at a time").
+//
+// A stable counting sort of the T*k assignments by expert in three kernels:
+//   dispatch_mask_kernel    one CTA per block of 256 tokens: a 256-bit token mask per
+//                           expert (atomicOr in shared memory) and its popcount;
+//   dispatch_scan_kernel    one CTA: per-expert totals, exclusive scan -> offsets, the
+//                           first packed row of every (block, expert), and the grouped
+//                           GEMM plan (active groups, tile prefixes);
+//   dispatch_scatter_kernel the packed row of assignment (t, j) is the block's base for
+//                           its expert plus the number of earlier tokens of the block in
+//                           the same mask -- token-ascending inside each expert, and the
+//                           same on every run.
+// An expert id outside [0, E) is skipped and raises the bounds flag in the status word.
+#include "device_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kPermBlock)
+dispatch_mask_kernel(const int32_t* __restrict__ ids, int T, int E, int k,
+                     uint32_t* __restrict__ blk_mask, int32_t* __restrict__ blk_count,
+                     uint32_t* __restrict__ status) {
+  extern __shared__ uint32_t mask[];  // [E][8]
+  const int b = blockIdx.x;
+  for (int i = threadIdx.x; i < E * 8; i += blockDim.x) mask[i] = 0;
+  __syncthreads();
+  const int i = threadIdx.x;
+  const int t = b * kPermBlock + i;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[(size_t)t * k + j];
+      if (e < 0 || e >= E) {
+        set_flag(status, kFlagBounds);
+        continue;
+      }
+      atomicOr(&mask[e * 8 + (i >> 5)], 1u << (i & 31));
+    }
+  }
+  __syncthreads();
+  uint32_t* gm = blk_mask + (size_t)b * E * 8;
+  for (int q = threadIdx.x; q < E * 8; q += blockDim.x) gm[q] = mask[q];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) c += __popc(mask[e * 8 + w]);
+    blk_count[(size_t)b * E + e] = c;
+  }
+}
+
+// Block-wide exclusive scan of one value per thread (blockDim.x == kScanThreads).
+__device__ int block_exclusive_scan(int v, int* smem_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) smem_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int s = smem_warp[lane];
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += n;
+    }
+    smem_warp[lane] = si - s;  // exclusive warp prefix
+    if (lane == 31) smem_warp[32] = si;
+  }
+  __syncthreads();
+  const int r = smem_warp[warp] + incl - v;
+  *total = smem_warp[32];
+  __syncthreads();
+  return r;
+}
+
+// Group sizes n_g (g < E routed, g == E shared = T) -> plan. Called by all threads of a
+// kScanThreads CTA; thread g handles group g (E + 1 <= 1025: thread 0 also takes E).
+__device__ void build_plan(const int* n_of, int E, int H, int I, int Is,
+                           PlanView pv, int* smem) {
+  // thread g takes group g (g <= E); with E == 1024 the last thread also takes group E
+  const int g = threadIdx.x;
+  int n0 = 0, n1 = 0, has1 = 0;
+  if (g <= E && g < kScanThreads) n0 = n_of[g];
+  if (g == kScanThreads - 1 && E == kScanThreads) { n1 = n_of[E]; has1 = 1; }
+  const int a0 = (g <= E && g < kScanThreads && n0 > 0) ? 1 : 0;
+  const int a1 = (has1 && n1 > 0) ? 1 : 0;
+  int tot;
+  const int pos = block_exclusive_scan(a0 + a1, smem, &tot);
+  if (a0) pv.active[pos] = g;
+  if (a1) pv.active[pos + a0] = E;
+  if (threadIdx.x == 0) *pv.n_active = tot;
+
+  auto inter = [&](int grp) { return grp < E ? I : Is; };
+  const int c0 = tc_nchunks(n0), c1 = tc_nchunks(n1);
+  const int t1a = (g <= E) ? c0 * (inter(g) / 128) : 0;
+  const int t1b = has1 ? c1 * (Is / 128) : 0;
+  const int t2a = (g <= E) ? c0 * (H / 256) : 0;
+  const int t2b = has1 ? c1 * (H / 256) : 0;
+  const int r0a = (g <= E) ? n0 : 0, r0b = has1 ? n1 : 0;
+  int tot1, tot2, totr;
+  const int p1 = block_exclusive_scan(t1a + t1b, smem, &tot1);
+  const int p2 = block_exclusive_scan(t2a + t2b, smem, &tot2);
+  const int pr = block_exclusive_scan(r0a + r0b, smem, &totr);
+  if (g <= E) {
+    pv.tp1[g] = p1;
+    pv.tp2[g] = p2;
+    pv.row0[g] = pr;
+  }
+  if (has1) {
+    pv.tp1[E] = p1 + t1a;
+    pv.tp2[E] = p2 + t2a;
+    pv.row0[E] = pr + r0a;
+  }
+  if (threadIdx.x == 0) {
+    pv.tp1[E + 1] = tot1;
+    pv.tp2[E + 1] = tot2;
+    pv.row0[E + 1] = totr;
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+dispatch_scan_kernel(const int32_t* blk_count, int nblk, int T, int E, int k, int H,
+                     int I, int Is, int32_t* blk_base, int32_t* __restrict__ offsets,
+                     int* __restrict__ plan_base) {
+  __shared__ int smem[33];
+  __shared__ int n_of[kMaxE + 1];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E) {
+    for (int b = 0; b < nblk; ++b) {
+      const int c = blk_count[(size_t)b * E + e];
+      blk_base[(size_t)b * E + e] = total;
+      total += c;
+    }
+  }
+  int R;
+  const int off = block_exclusive_scan(e < E ? total : 0, smem, &R);
+  if (e < E) {
+    offsets[e] = off;
+    for (int b = 0; b < nblk; ++b) blk_base[(size_t)b * E + e] += off;
+    n_of[e] = total;
+  }
+  if (threadIdx.x == 0) {
+    offsets[E] = R;
+    n_of[E] = T;
+  }
+  __syncthreads();
+  build_plan(n_of, E, H, I, Is, plan_view(plan_base, E), smem);
+}
+
+__global__ void __launch_bounds__(kPermBlock)
+dispatch_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T,
+                        int E, int k, const uint32_t* __restrict__ blk_mask,
+                        const int32_t* __restrict__ blk_base, int32_t* __restrict__ sorted_token,
+                        float* __restrict__ sorted_w, int32_t* __restrict__ assign_row) {
+  const int b = blockIdx.x;
+  const int i = threadIdx.x;
+  const int t = b * kPermBlock + i;
+  if (t >= T) return;
+  const uint32_t* gm = blk_mask + (size_t)b * E * 8;
+  const int word = i >> 5;
+  const uint32_t below = (1u << (i & 31)) - 1u;
+  for (int j = 0; j < k; ++j) {
+    const int e = ids[(size_t)t * k + j];
+    if (e < 0 || e >= E) continue;
+    const uint32_t* m = gm + e * 8;
+    int rank = __popc(m[word] & below);
+    for (int w = 0; w < word; ++w) rank += __popc(m[w]);
+    const int p = blk_base[(size_t)b * E + e] + rank;
+    sorted_token[p] = t;
+    if (sorted_w) sorted_w[p] = topk_w[(size_t)t * k + j];
+    assign_row[(size_t)t * k + j] = p;
+  }
+}
+
+// Plan from caller-supplied offsets. Offsets that are not a monotone partition of at most
+// T*k rows starting at 0 are flagged and give an empty plan (no GEMM work).
+__global__ void __launch_bounds__(kScanThreads)
+plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int T, int E, int k, int H, int I,
+                         int Is, int* __restrict__ plan_base, uint32_t* __restrict__ status) {
+  __shared__ int smem[33];
+  __shared__ int n_of[kMaxE + 1];
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = (offsets[0] != 0 || offsets[E] > T * k) ? 1 : 0;
+  __syncthreads();
+  for (int g = threadIdx.x; g < E; g += blockDim.x) {
+    const int n = offsets[g + 1] - offsets[g];
+    if (n < 0) bad = 1;
+    n_of[g] = n;
+  }
+  if (threadIdx.x == 0) n_of[E] = T;
+  __syncthreads();
+  if (bad) {
+    for (int g = threadIdx.x; g <= E; g += blockDim.x) n_of[g] = 0;
+    if (threadIdx.x == 0) set_flag(status, kFlagBounds);
+  }
+  __syncthreads();
+  build_plan(n_of, E, H, I, Is, plan_view(plan_base, E), smem);
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const moe_shape& s, const Layout& L, char* ws, const int32_t* ids,
+                           const float* topk_w, int32_t* offsets, int32_t* sorted_token,
+                           float* sorted_w, int32_t* assign_row, cudaStream_t st) {
+  LaunchScope scope(MOE_K_PERMUTE, st, 3);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  uint32_t* blk_mask = reinterpret_cast<uint32_t*>(ws + L.blk_mask);
+  int32_t* blk_base = reinterpret_cast<int32_t*>(ws + L.blk_base);
+  const size_t smem = (size_t)s.E * 8 * sizeof(uint32_t);
+  // counts go to blk_base first, the scan rewrites them in place as bases
+  dispatch_mask_kernel<<<L.nblk, kPermBlock, smem, st>>>(ids, s.T, s.E, s.k, blk_mask, blk_base,
+                                                        status);
+  dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(blk_base, L.nblk, s.T, s.E, s.k, s.H, s.I, s.Is,
+                                                   blk_base, offsets,
+                                                   reinterpret_cast<int*>(ws + L.plan));
+  dispatch_scatter_kernel<<<L.nblk, kPermBlock, 0, st>>>(ids, topk_w, s.T, s.E, s.k, blk_mask,
+                                                         blk_base, sorted_token, sorted_w,
+                                                         assign_row);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_plan_from_offsets(const moe_shape& s, const Layout& L, char* ws,
+                                     const int32_t* offsets, cudaStream_t st) {
+  LaunchScope scope(MOE_K_PERMUTE, st);
+  plan_from_offsets_kernel<<<1, kScanThreads, 0, st>>>(
+      offsets, s.T, s.E, s.k, s.H, s.I, s.Is, reinterpret_cast<int*>(ws + L.plan),
+      reinterpret_cast<uint32_t*>(ws + L.status));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

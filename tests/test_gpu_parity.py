@@ -1,0 +1,372 @@
+"""GPU parity of every stage of the layer against the fp64 oracle, through the C ABI.
+
+Inputs come from the seeded generator (device half on the GPU, host half for the
+oracle; a test checks they are bit-identical). The tolerance is the layer's:
+max |gpu - ref| <= 1e-2 RMS(ref), mean relative error <= 2e-3; routing id sets exact
+except near-ties (10th/11th fp64 logit gap < 1e-5). Integer dispatch: bit-exact.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU, skipped there
+    pytestmark = pytest.mark.skip(reason="needs a CUDA device")
+
+import oracle  # noqa: E402
+import sparse_moe_expert_fp32_b200 as moe  # noqa: E402
+import synth  # noqa: E402
+from parity_util import NEAR_TIE_GAP, assert_layer_close, err_stats, id_sets_match  # noqa: E402
+
+VARIANTS = {"stream": moe.MOE_VARIANT_STREAM}
+
+
+def _u16(t):
+    """bf16 torch tensor -> numpy uint16 bits."""
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _dev_i32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+
+def _dev_f32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+@pytest.fixture(autouse=True)
+def _variant_reset():
+    yield
+    moe.moe_set_variant(moe.MOE_VARIANT_AUTO)
+
+
+def _forward(cfg, dev, variant=None, seed_ws=True):
+    if variant is not None:
+        moe.moe_set_variant(variant)
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s)
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device="cuda")
+    gap = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
+    moe.moe_layer_forward(s, dev["x"], dev, out, ws, topk_ids=ids, topk_w=tw, gap=gap)
+    st, flags = moe.moe_device_status(ws)
+    assert st == moe.MOE_OK, (st, flags)
+    return out.cpu().numpy(), ids.cpu().numpy(), tw.cpu().numpy(), gap.cpu().numpy()
+
+
+def _check_layer(cfg, host, out, ids, rows):
+    """Oracle on token rows `rows`; ids exact except near-ties, outputs within tolerance."""
+    ref = oracle.forward_inputs(host, rows=rows)
+    differ = id_sets_match(ids[rows], ref["ids"], ref["gap"], ref["logits"])
+    keep = [i for i in range(len(rows)) if i not in set(differ)]
+    stats = assert_layer_close(out[rows][keep], ref["out"][keep], cfg.name)
+    return stats, len(differ)
+
+
+# ----------------------------------------------------------------------------- generator
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["tiny", "t24_skewed"])
+def test_generator_device_equals_host(name):
+    cfg = synth.CONFIGS[name]
+    if name == "t24_skewed":
+        cfg = cfg.replace(T=64, E=8)  # same recipe (zero rows, Zipf bias), few experts
+    dev = synth.device_inputs(cfg, seed=1)
+    host = synth.host_inputs(cfg, seed=1)
+    assert np.array_equal(_u16(dev["x"]), host.x)
+    assert np.array_equal(dev["w_router"].cpu().numpy(), host.w_router)
+    assert np.array_equal(_u16(dev["w_gate_up"]), host.gate_up_all())
+    assert np.array_equal(_u16(dev["w_down"]), host.down_all())
+    assert np.array_equal(_u16(dev["ws_gate_up"]), host.ws_gate_up)
+    assert np.array_equal(_u16(dev["ws_down"]), host.ws_down)
+    assert np.array_equal(_u16(dev["w_shared_gate"]), host.w_shared_gate)
+    if host.router_bias is not None:
+        assert np.array_equal(dev["router_bias"].cpu().numpy(), host.router_bias)
+
+
+# ----------------------------------------------------------------------------- router
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", sorted(synth.CONFIGS))
+def test_router_topk_parity(name):
+    cfg = synth.CONFIGS[name]
+    dev = synth.device_inputs(cfg, seed=0)
+    host = synth.host_inputs(cfg, seed=0)
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s)
+    ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device="cuda")
+    sg = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
+    gap = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
+    moe.moe_router_topk(s, dev["x"], dev, ids, tw, sg, gap, ws)
+    torch.cuda.synchronize()
+    logits = oracle.router_logits(host.x, host.w_router, host.router_bias)
+    rids, rgap = oracle.topk_select(logits, cfg.k)
+    gids = ids.cpu().numpy()
+    differ = id_sets_match(gids, rids, rgap, logits)
+    assert len(differ) <= max(4, cfg.T // 1000), differ
+    same = [t for t in range(cfg.T) if t not in set(differ)]
+    rw = oracle.routing_weights(logits, rids)
+    # order inside a token: descending logit; compare weights by expert id
+    gw = tw.cpu().numpy()
+    for t in same[:: max(1, len(same) // 2000)]:
+        a = dict(zip(gids[t].tolist(), gw[t].tolist()))
+        b = dict(zip(rids[t].tolist(), rw[t].tolist()))
+        for e in b:
+            assert abs(a[e] - b[e]) <= 1e-5 + 1e-4 * b[e], (t, e, a[e], b[e])
+    assert np.allclose(gw.sum(axis=1), 1.0, atol=1e-5)
+    rsg = oracle.shared_gate(host.x, host.w_shared_gate)
+    assert np.allclose(sg.cpu().numpy(), rsg, rtol=1e-5, atol=1e-6)
+    g = gap.cpu().numpy()
+    assert (g >= 0).all()
+    assert np.allclose(g[same], rgap[same], atol=5e-5)
+
+
+@pytest.mark.gpu
+def test_router_ties_go_to_lower_index():
+    cfg = synth.CONFIGS["tiny"].replace(T=40)
+    dev = synth.device_inputs(cfg, seed=3)
+    wr = dev["w_router"]
+    wr[9] = wr[2]   # experts 2 and 9 tie exactly
+    wr[15] = wr[0]  # experts 0 and 15 tie exactly
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s)
+    ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device="cuda")
+    sg = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
+    moe.moe_router_topk(s, dev["x"], dev, ids, tw, sg, None, ws)
+    host_wr = wr.cpu().numpy()
+    x = _u16(dev["x"])
+    logits = oracle.router_logits(x, host_wr)
+    rids, _ = oracle.topk_select(logits, cfg.k)
+    gids = ids.cpu().numpy()
+    for t in range(cfg.T):
+        assert set(gids[t]) == set(rids[t]), t
+        if 9 in gids[t]:
+            assert 2 in gids[t]
+        if 15 in gids[t]:
+            assert 0 in gids[t]
+
+
+# ----------------------------------------------------------------------------- dispatch
+
+def _random_ids(T, E, k, seed, hot=None):
+    rng = np.random.default_rng(seed)
+    ids = np.empty((T, k), dtype=np.int32)
+    for t in range(T):
+        if hot is not None:
+            rest = rng.choice(np.setdiff1d(np.arange(E), [hot]), k - 1, replace=False)
+            ids[t] = np.concatenate([[hot], rest])
+        else:
+            ids[t] = rng.choice(E, k, replace=False)
+    return ids
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,E,k,hot", [(64, 16, 4, None), (1, 512, 10, None), (257, 512, 10, None),
+                                       (8192, 512, 10, None), (1000, 64, 8, 5), (300, 1024, 32, None),
+                                       (5, 4, 4, None)])
+def test_permute_bitexact(T, E, k, hot):
+    ids = _random_ids(T, E, k, seed=T + E, hot=hot)
+    s = moe.make_shape(T, 256, E, k, 128, 128)
+    ws = moe.alloc_workspace(s)
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    st = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    ar = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    moe.moe_permute(s, _dev_i32(ids), off, st, ar, ws)
+    r_off, r_st, r_ar, _ = oracle.permute(ids, E)
+    assert np.array_equal(off.cpu().numpy(), r_off)
+    assert np.array_equal(st.cpu().numpy(), r_st)
+    assert np.array_equal(ar.cpu().numpy().reshape(T, k), r_ar)
+    assert moe.moe_device_status(ws)[0] == moe.MOE_OK
+
+
+@pytest.mark.gpu
+def test_permute_flags_out_of_range_ids():
+    T, E, k = 32, 16, 4
+    ids = _random_ids(T, E, k, seed=1)
+    ids[5, 2] = E + 3
+    ids[9, 0] = -1
+    s = moe.make_shape(T, 256, E, k, 128, 128)
+    ws = moe.alloc_workspace(s)
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    st = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    ar = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    moe.moe_permute(s, _dev_i32(ids), off, st, ar, ws)
+    status, flags = moe.moe_device_status(ws)
+    assert status == moe.MOE_ERR_DEVICE_BOUNDS and flags & 1
+    assert off.cpu().numpy()[-1] == T * k - 2  # the two bad assignments were skipped
+    assert moe.moe_device_status(ws)[0] == moe.MOE_OK  # cleared
+
+
+# ----------------------------------------------------------------------------- grouped GEMMs
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
+@pytest.mark.parametrize("name", ["tiny", "flash_decode"])
+def test_grouped_swiglu_and_combine_staged(name, variant):
+    cfg = synth.CONFIGS[name]
+    moe.moe_set_variant(VARIANTS[variant])
+    dev = synth.device_inputs(cfg, seed=0)
+    host = synth.host_inputs(cfg, seed=0)
+    ref = oracle.forward_inputs(host)
+    ids = ref["ids"]  # oracle routing drives both sides
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s)
+    R = cfg.R
+    off = torch.empty(cfg.E + 1, dtype=torch.int32, device="cuda")
+    st = torch.empty(R, dtype=torch.int32, device="cuda")
+    ar = torch.empty(R, dtype=torch.int32, device="cuda")
+    moe.moe_permute(s, _dev_i32(ids), off, st, ar, ws)
+    y = torch.full((R, cfg.H), float("nan"), dtype=torch.float32, device="cuda")
+    ys = torch.full((cfg.T, cfg.H), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_grouped_swiglu(s, dev["x"], st, off, dev, y, ys, ws)
+    yref = oracle.expert_outputs_packed(host.x, ids, host.gate_up, host.down, cfg.E)
+    assert_layer_close(y.cpu().numpy(), yref, "y")
+    assert_layer_close(ys.cpu().numpy(), ref["shared"], "y_shared")
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    moe.moe_unpermute_combine(s, y, ys, ar, _dev_f32(ref["weights"]), _dev_f32(ref["shared_gate"]), out)
+    assert_layer_close(out.cpu().numpy(), ref["out"], "combined")
+    assert moe.moe_device_status(ws)[0] == moe.MOE_OK
+
+
+@pytest.mark.gpu
+def test_combine_exact_inputs():
+    rng = np.random.default_rng(7)
+    T, H, k, E = 37, 320, 6, 20
+    R = T * k
+    y = rng.standard_normal((R, H)).astype(np.float32)
+    ysh = rng.standard_normal((T, H)).astype(np.float32)
+    ar = rng.permutation(R).astype(np.int32).reshape(T, k)
+    w = rng.random((T, k)).astype(np.float32)
+    sg = rng.random(T).astype(np.float32)
+    s = moe.make_shape(T, H, E, k, 64, 64)
+    out = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    moe.moe_unpermute_combine(s, _dev_f32(y), _dev_f32(ysh), _dev_i32(ar), _dev_f32(w), _dev_f32(sg), out)
+    ref = oracle.combine(y, ysh, ar, w, sg)
+    assert np.allclose(out.cpu().numpy(), ref, rtol=1e-5, atol=1e-5)
+
+
+# ----------------------------------------------------------------------------- whole layer
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
+@pytest.mark.parametrize("name", ["tiny", "flash_decode"])
+def test_layer_forward_full(name, variant):
+    cfg = synth.CONFIGS[name]
+    dev = synth.device_inputs(cfg, seed=0)
+    host = synth.host_inputs(cfg, seed=0)
+    out, ids, _, _ = _forward(cfg, dev, VARIANTS[variant])
+    stats, ties = _check_layer(cfg, host, out, ids, list(range(cfg.T)))
+    print(name, variant, stats, "near-ties", ties)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
+@pytest.mark.parametrize("name,nsample", [("flash_prefill", 96), ("t24_prefill", 6), ("t24_skewed", 8)])
+def test_layer_forward_sampled(name, nsample, variant):
+    cfg = synth.CONFIGS[name]
+    dev = synth.device_inputs(cfg, seed=0)
+    out, ids, _, _ = _forward(cfg, dev, VARIANTS[variant])
+    del dev
+    torch.cuda.empty_cache()
+    host = synth.host_inputs(cfg, seed=0)
+    rng = np.random.default_rng(123)
+    rows = sorted(set([0, cfg.T - 1] + rng.choice(cfg.T, nsample, replace=False).tolist()))
+    stats, ties = _check_layer(cfg, host, out, ids, rows)
+    print(name, variant, stats, "near-ties", ties)
+
+
+EDGE = {
+    "T1": dict(T=1),
+    "T3_ragged": dict(T=3),
+    "T257_blocks": dict(T=257),
+    "k1": dict(k=1),
+    "E_eq_k": dict(E=4, k=4),
+    "E1": dict(E=1, k=1),
+    "shared_narrower": dict(Is=64, I=128),
+    "H64_I64": dict(H=64, I=64, Is=64),
+    "max_E_k": dict(T=40, E=1024, k=32),
+}
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
+@pytest.mark.parametrize("case", sorted(EDGE))
+def test_layer_edge_cases(case, variant):
+    cfg = synth.CONFIGS["tiny"].replace(name=case, **EDGE[case])
+    dev = synth.device_inputs(cfg, seed=5)
+    host = synth.host_inputs(cfg, seed=5)
+    out, ids, tw, _ = _forward(cfg, dev, VARIANTS[variant])
+    _check_layer(cfg, host, out, ids, list(range(cfg.T)))
+    if cfg.k == 1:
+        assert (tw == 1.0).all()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
+def test_hot_expert_many_tokens(variant):
+    """A router bias sends every token to expert 3: 600 rows in one group (several tiles)."""
+    cfg = synth.CONFIGS["tiny"].replace(name="hot", T=600)
+    dev = synth.device_inputs(cfg, seed=6)
+    bias = np.zeros(cfg.E, np.float32)
+    bias[3] = 50.0
+    dev["router_bias"] = _dev_f32(bias)
+    host = synth.host_inputs(cfg, seed=6)
+    host.router_bias = bias
+    out, ids, _, _ = _forward(cfg, dev, VARIANTS[variant])
+    assert (ids == 3).any(axis=1).all()
+    _check_layer(cfg, host, out, ids, list(range(cfg.T)))
+
+
+@pytest.mark.gpu
+def test_empty_batch_and_host_entry():
+    cfg = synth.CONFIGS["tiny"]
+    dev = synth.device_inputs(cfg, seed=0)
+    s0 = moe.shape_of(cfg, T=0)
+    ws0 = moe.alloc_workspace(s0)
+    moe.moe_layer_forward(s0, dev["x"], dev, torch.empty(16, device="cuda"), ws0)
+    # host entry point: pinned host x -> device -> pinned host out
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s, host_staging=True)
+    x_host = dev["x"].cpu().pin_memory()
+    out_host = torch.empty((cfg.T, cfg.H), dtype=torch.float32).pin_memory()
+    moe.moe_layer_forward_host(s, x_host, dev, out_host, ws)
+    torch.cuda.synchronize()
+    out_dev, _, _, _ = _forward(cfg, dev)
+    st = err_stats(out_host.numpy(), out_dev)
+    assert st["max_abs_over_rms"] < 1e-5
+
+
+@pytest.mark.gpu
+def test_bounded_wait_reports_timeout():
+    ws = moe.alloc_workspace(moe.shape_of(synth.CONFIGS["tiny"]))
+    flag = torch.zeros(4, dtype=torch.int32, device="cuda")  # nothing ever sets it
+    moe.moe_debug_wait_flag(flag, 2_000_000, ws)  # 2 ms
+    status, flags = moe.moe_device_status(ws)
+    assert status == moe.MOE_ERR_DEVICE_TIMEOUT and flags & 2
+    flag.fill_(1)
+    moe.moe_debug_wait_flag(flag, 2_000_000, ws)
+    assert moe.moe_device_status(ws)[0] == moe.MOE_OK
+
+
+@pytest.mark.gpu
+def test_profile_and_launch_count():
+    cfg = synth.CONFIGS["tiny"]
+    dev = synth.device_inputs(cfg, seed=0)
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s)
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    moe.moe_profile_enable(True)
+    n0 = moe.moe_launch_count()
+    moe.moe_layer_forward(s, dev["x"], dev, out, ws)
+    n1 = moe.moe_launch_count()
+    moe.moe_profile_enable(False)
+    prof = moe.moe_profile_collect()
+    assert n1 - n0 >= 5
+    assert prof["gate_up"][1] == 1 and prof["down"][1] == 1 and prof["gate_up"][0] > 0
+
+
+def test_near_tie_threshold_constant():
+    assert NEAR_TIE_GAP == 1e-5
