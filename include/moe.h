@@ -138,7 +138,8 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_ids, int32_t*
  *   y[p,:]        = expert_{e(p)}(x[sorted_token[p],:])   fp32 [T*k][H] (packed order)
  *   y_shared[t,:] = shared(x[t,:])                         fp32 [T][H]
  * sorted_token / offsets as produced by moe_permute. The intermediate
- * h = SiLU(gate) * up is rounded to bf16 before the down projection; accumulation is fp32.
+ * h = SiLU(gate) * up is carried as a pair of bf16 values (hi = bf16(h), lo = bf16(h - hi),
+ * about 16 significant bits) into the down projection; accumulation is fp32.
  */
 moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const int32_t* sorted_token,
                               const int32_t* offsets, const moe_weights* weights, float* y,

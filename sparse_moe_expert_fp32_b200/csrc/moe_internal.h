@@ -35,7 +35,9 @@ struct Layout {
   size_t sorted_w;      // fp32 [T*k]: routing weight of each packed row
   size_t assign_row;    // int32 [T*k]
   size_t plan;          // int32 plan arrays (see PlanView)
-  size_t h;             // bf16 [T*k + T][ldh]: SwiGLU intermediate, routed rows then shared rows
+  size_t h;             // bf16 [2][T*k + T][ldh]: SwiGLU intermediate as a hi|lo pair of planes
+                        // (h = hi + lo), routed rows then shared rows
+  size_t h_plane;       // elements per plane: (T*k + T) * ldh
   size_t total;
   int nblk;
   int ldh;              // max(I, Is)
@@ -66,9 +68,13 @@ __host__ __device__ inline PlanView plan_view(void* base, int E) {
   return v;
 }
 
-// Tensor-core tiling of group g with n rows: ceil(n/256) token chunks, split evenly
-// into chunks that are multiples of 16 rows.
-__host__ __device__ inline int tc_nchunks(int n) { return (n + kTcChunk - 1) / kTcChunk; }
+// Tensor-core tiling of a group with n rows into ceil(n / max) token chunks of nearly equal
+// size (multiples of 16 rows): max 256 rows for the gate|up GEMM, 128 for the down GEMM
+// (whose B operand holds the hi and lo rows of each token).
+constexpr int kTcChunkDown = 128;
+__host__ __device__ inline int tc_nchunks(int n, int max_rows) {
+  return (n + max_rows - 1) / max_rows;
+}
 
 // ---------------------------------------------------------------- launch bookkeeping
 

@@ -99,11 +99,12 @@ __device__ void build_plan(const int* n_of, int E, int H, int I, int Is,
   if (threadIdx.x == 0) *pv.n_active = tot;
 
   auto inter = [&](int grp) { return grp < E ? I : Is; };
-  const int c0 = tc_nchunks(n0), c1 = tc_nchunks(n1);
+  const int c0 = tc_nchunks(n0, kTcChunk), c1 = tc_nchunks(n1, kTcChunk);
+  const int d0 = tc_nchunks(n0, kTcChunkDown), d1 = tc_nchunks(n1, kTcChunkDown);
   const int t1a = (g <= E) ? c0 * (inter(g) / 128) : 0;
   const int t1b = has1 ? c1 * (Is / 128) : 0;
-  const int t2a = (g <= E) ? c0 * (H / 256) : 0;
-  const int t2b = has1 ? c1 * (H / 256) : 0;
+  const int t2a = (g <= E) ? d0 * (H / 256) : 0;
+  const int t2b = has1 ? d1 * (H / 256) : 0;
   const int r0a = (g <= E) ? n0 : 0, r0b = has1 ? n1 : 0;
   int tot1, tot2, totr;
   const int p1 = block_exclusive_scan(t1a + t1b, smem, &tot1);

@@ -8,8 +8,9 @@
 // with 16-byte loads (no L1 allocation) and applies them to up to 4 tokens held in
 // registers; 32 partial sums are combined by one warp transpose-reduction.
 //
-//   stream_gate_up_kernel : h[p, c] = bf16( SiLU(gate_c . x_p) * (up_c . x_p) )
-//   stream_down_kernel    : y[p, m] = W_down[m, :] . h[p, :]; stored per packed row, or
+//   stream_gate_up_kernel : h[p, c] = SiLU(gate_c . x_p) * (up_c . x_p), kept as the bf16
+//                           pair hi = bf16(h), lo = bf16(h - hi) (about 16 significant bits)
+//   stream_down_kernel    : y[p, m] = W_down[m, :] . (hi + lo)[p, :]; stored per packed row, or
 //                           scaled by the routing weight (shared gate for the shared
 //                           expert) and added into out[token, m] ("Weighted combine").
 #include "device_common.cuh"
@@ -40,8 +41,9 @@ __device__ __forceinline__ int token_of(const int32_t* sorted_token, int p, int 
 __global__ void __launch_bounds__(kWarps * 32)
 stream_gate_up_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_token,
                       const int* __restrict__ plan_base, const uint16_t* __restrict__ w_gate_up,
-                      const uint16_t* __restrict__ ws_gate_up, uint16_t* __restrict__ h, int T,
-                      int H, int E, int I, int Is, int ldh, uint32_t* __restrict__ status) {
+                      const uint16_t* __restrict__ ws_gate_up, uint16_t* __restrict__ h,
+                      size_t h_plane, int T, int H, int E, int I, int Is, int ldh,
+                      uint32_t* __restrict__ status) {
   const PlanView pv = plan_view(const_cast<int*>(plan_base), E);
   const int gi = blockIdx.y;
   if (gi >= *pv.n_active) return;
@@ -92,14 +94,18 @@ stream_gate_up_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict_
     if (lane < 16 && s + q < n) {
       const float gate = v;
       const float hv = gate / (1.f + expf(-gate)) * up;
-      h[(size_t)(row0 + s + q) * ldh + c0 + (lane >> 2)] = f32_to_bf16_rn(hv);
+      const uint16_t hi = f32_to_bf16_rn(hv);
+      const size_t at = (size_t)(row0 + s + q) * ldh + c0 + (lane >> 2);
+      h[at] = hi;
+      h[h_plane + at] = f32_to_bf16_rn(hv - bf16lo(hi));
     }
   }
 }
 
 // grid: (H / 64, E + 1)
 __global__ void __launch_bounds__(kWarps * 32)
-stream_down_kernel(const uint16_t* __restrict__ h, const int32_t* __restrict__ sorted_token,
+stream_down_kernel(const uint16_t* __restrict__ h, size_t h_plane,
+                   const int32_t* __restrict__ sorted_token,
                    const float* __restrict__ sorted_w, const float* __restrict__ sgate,
                    const int* __restrict__ plan_base, const uint16_t* __restrict__ w_down,
                    const uint16_t* __restrict__ ws_down, float* __restrict__ y,
@@ -132,8 +138,11 @@ stream_down_kernel(const uint16_t* __restrict__ h, const int32_t* __restrict__ s
       for (int r = 0; r < 8; ++r) wv[r] = ld_stream_v4(W + (size_t)(m0 + r) * Ig + 8 * c);
 #pragma unroll
       for (int q = 0; q < kTok; ++q) {
-        float hf[8];
+        float hf[8], lf[8];
         unpack8(ld_v4(hrow[q] + 8 * c), hf);
+        unpack8(ld_v4(hrow[q] + h_plane + 8 * c), lf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hf[i] += lf[i];
 #pragma unroll
         for (int r = 0; r < 8; ++r) acc[r * 4 + q] = dot8_acc(wv[r], hf, acc[r * 4 + q]);
       }
@@ -167,7 +176,7 @@ cudaError_t launch_stream_gate_up(const moe_shape& s, const Layout& L, char* ws,
   stream_gate_up_kernel<<<grid, kWarps * 32, 0, st>>>(
       x, sorted_token, reinterpret_cast<const int*>(ws + L.plan),
       static_cast<const uint16_t*>(w.w_gate_up), static_cast<const uint16_t*>(w.ws_gate_up),
-      reinterpret_cast<uint16_t*>(ws + L.h), s.T, s.H, s.E, s.I, s.Is, L.ldh,
+      reinterpret_cast<uint16_t*>(ws + L.h), L.h_plane, s.T, s.H, s.E, s.I, s.Is, L.ldh,
       reinterpret_cast<uint32_t*>(ws + L.status));
   return cudaGetLastError();
 }
@@ -179,7 +188,7 @@ cudaError_t launch_stream_down(const moe_shape& s, const Layout& L, char* ws,
   LaunchScope scope(MOE_K_DOWN, st);
   dim3 grid((s.H + kWarps * kRowsDown - 1) / (kWarps * kRowsDown), s.E + 1);
   stream_down_kernel<<<grid, kWarps * 32, 0, st>>>(
-      reinterpret_cast<const uint16_t*>(ws + L.h), sorted_token, sorted_w, sgate,
+      reinterpret_cast<const uint16_t*>(ws + L.h), L.h_plane, sorted_token, sorted_w, sgate,
       reinterpret_cast<const int*>(ws + L.plan), static_cast<const uint16_t*>(w.w_down),
       static_cast<const uint16_t*>(w.ws_down), y, y_shared, out, s.T, s.H, s.E, s.I, s.Is, L.ldh,
       reinterpret_cast<uint32_t*>(ws + L.status));
