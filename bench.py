@@ -49,7 +49,8 @@ KERNEL_SOURCES = {  # kernel id -> source file whose hash a stored ncu traffic f
     "combine": ("combine.cu",),
 }
 # oracle token sample per workload for the CPU baseline (about 10-30 s on a host)
-CPU_SAMPLE = {"tiny": 64, "flash_decode": 16, "flash_prefill": 32, "t24_prefill": 3, "t24_skewed": 3}
+CPU_SAMPLE = {"tiny": 64, "flash_decode": 16, "flash_prefill": 32, "flash_prefill_e64": 32,
+              "t24_prefill": 3, "t24_skewed": 3}
 
 
 def log(*a):
@@ -128,10 +129,10 @@ class ClockSampler:
 def algorithmic_bytes(kernel: str, cfg, n_active: int) -> float:
     """Bytes a launch of `kernel` must move at least (each operand once)."""
     T, H, I, Is, R = cfg.T, cfg.H, cfg.I, cfg.Is, cfg.R
-    if kernel == "gate_up":  # activated experts' gate|up + shared gate|up + x + h
-        return (n_active * 2 * I * H + 2 * Is * H + T * H) * 2 + (R * I + T * Is) * 2
-    if kernel == "down":  # activated experts' down + shared down + h in + out (fp32)
-        return (n_active * H * I + H * Is) * 2 + (R * I + T * Is) * 2 + T * H * 4
+    if kernel == "gate_up":  # activated experts' gate|up + shared gate|up + x + h (hi+lo bf16)
+        return (n_active * 2 * I * H + 2 * Is * H + T * H) * 2 + (R * I + T * Is) * 4
+    if kernel == "down":  # activated experts' down + shared down + h (hi+lo) in + out (fp32)
+        return (n_active * H * I + H * Is) * 2 + (R * I + T * Is) * 4 + T * H * 4
     if kernel == "router_logits":
         return cfg.E * H * 4 + T * H * 2 + T * cfg.E * 4
     if kernel == "router_topk":

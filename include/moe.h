@@ -72,9 +72,11 @@ typedef struct moe_weights {
 
 /* Grouped-GEMM variant used by moe_grouped_swiglu and moe_layer_forward. */
 typedef enum moe_variant {
-  MOE_VARIANT_AUTO = 0,   /* streaming when T*k/E < 16 tokens per expert, else tensor-core */
-  MOE_VARIANT_STREAM = 1, /* weight-streaming CUDA-core kernels (decode-size batches)      */
-  MOE_VARIANT_TC = 2      /* tcgen05/TMEM grouped GEMMs fed by TMA (prefill)               */
+  MOE_VARIANT_AUTO = 0,   /* tensor-core kernels where the shape allows (I, Is multiples of
+                             128, H of 256), else the streaming kernels                    */
+  MOE_VARIANT_STREAM = 1, /* weight-streaming CUDA-core kernels                             */
+  MOE_VARIANT_TC = 2      /* tcgen05/TMEM grouped GEMMs fed by TMA (falls back to streaming
+                             for shapes they do not support)                               */
 } moe_variant;
 
 /* Kernel ids for the measurement calls below. */

@@ -137,13 +137,13 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
   } while (0)
 #define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
 
-// Tensor-core variant for this shape? AUTO: when there are at least 16 rows per expert.
+// Tensor-core variant for this shape? AUTO takes it wherever the shape allows: on B200 it
+// streams the activated experts' weights faster than the CUDA-core kernels even at
+// decode sizes (a 16-token MMA tile costs nothing next to the weight bytes).
 bool use_tc(const moe_shape& s) {
   const int v = g_variant.load();
   if (v == MOE_VARIANT_STREAM) return false;
-  if (!tc_supported(s)) return false;
-  if (v == MOE_VARIANT_TC) return true;
-  return (int64_t)s.T * s.k >= 16 * (int64_t)s.E;
+  return tc_supported(s);
 }
 
 // Stage 4 on the plan in the workspace: fused (out != NULL) or per-row y / y_shared.

@@ -3,7 +3,9 @@
 // normalises the selected router probabilities; the shared expert has its own sigmoid
 // output gate).
 //
-//   router_logits_stream_kernel : logits = x . Wr^T on CUDA cores, fp32 accumulation.
+//   router_logits_stream_kernel : logits = x . Wr^T on CUDA cores, fp32 accumulation
+//                                 (small batches; larger ones use the tensor-core router
+//                                 in tc_gemm.cu).
 //   router_topk_kernel          : one warp per token: top-k with lowest-index ties,
 //                                 renormalised softmax weights, 10th/11th gap,
 //                                 shared-expert gate sigmoid(w_shared . x).
@@ -11,6 +13,7 @@
 
 #include "device_common.cuh"
 #include "moe_internal.h"
+#include "tc_gemm.h"
 
 namespace moe {
 namespace {
@@ -172,10 +175,14 @@ cudaError_t launch_router_logits_stream(const moe_shape& s, const uint16_t* x, c
   return cudaGetLastError();
 }
 
+// Token count from which the tensor-core router (a GEMM over the exact three-piece split
+// of the router matrix) replaces the CUDA-core one.
+constexpr int kTcRouterMinTokens = 512;
+
 cudaError_t launch_router_logits(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                                  const float* wr, float* logits, cudaStream_t st) {
-  (void)L;
-  (void)ws;
+  if (s.T >= kTcRouterMinTokens && tc_router_supported(s))
+    return launch_tc_router(s, L, ws, x, wr, logits, st);
   return launch_router_logits_stream(s, x, wr, logits, st);
 }
 

@@ -27,6 +27,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "device_common.cuh"
@@ -46,7 +47,7 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcc1Col = 256;  // column of the second accumulator
 
-enum Mode { kGateUp = 0, kDown = 1 };
+enum Mode { kGateUp = 0, kDown = 1, kRouter = 2 };
 
 struct SharedState {
   uint64_t full[kStages];
@@ -73,6 +74,8 @@ struct TcArgs {
   float* y_shared;
   float* out;
   uint32_t* status;
+  float* logits;  // router: [T][E]
+  int ntiles;     // router: tile count (no plan)
 };
 
 struct Tile {
@@ -142,6 +145,50 @@ __device__ __forceinline__ int token_of_row(const TcArgs& a, int p, int R) {
   return t;
 }
 
+// Everything the three roles need to know about one tile.
+struct Geom {
+  Tile t;
+  int a_row0, a_row1;  // A-operand rows of the two accumulators
+  int nk;              // 64-wide K steps
+  bool shared;         // shared-expert group (its own weight tensor map)
+};
+
+template <int MODE>
+__device__ __forceinline__ Geom tile_geom(const TcArgs& a, const PlanView& pv, int tile) {
+  Geom G;
+  if (MODE == kRouter) {
+    // 256 router rows (experts) x up to 256 tokens; K runs over the hi|mid|lo pieces
+    const int mt = (a.E + 255) / 256;
+    const int m = tile % mt, c = tile / mt;
+    G.t.g = 0;
+    G.t.m = m;
+    G.t.p0 = c * 256;
+    G.t.nvalid = min(256, a.T - G.t.p0);
+    G.t.N = (G.t.nvalid + 15) & ~15;
+    G.a_row0 = m * 256;
+    G.a_row1 = m * 256 + 128;
+    G.nk = 3 * a.H / 64;
+    G.shared = false;
+    return G;
+  }
+  const int* tp = (MODE == kGateUp) ? pv.tp1 : pv.tp2;
+  G.t = decode_tile(pv, tp, a.E, tile, (MODE == kGateUp) ? kTcChunk : kTcChunkDown);
+  G.shared = G.t.g == a.E;
+  if (MODE == kGateUp) {
+    const int Ig = G.shared ? a.Is : a.I;
+    const int base = G.shared ? 0 : G.t.g * 2 * a.I;
+    G.a_row0 = base + G.t.m * 128;
+    G.a_row1 = base + Ig + G.t.m * 128;
+    G.nk = a.H / 64;
+  } else {
+    const int base = G.shared ? 0 : G.t.g * a.H;
+    G.a_row0 = base + G.t.m * 256;
+    G.a_row1 = G.a_row0 + 128;
+    G.nk = (G.shared ? a.Is : a.I) / 64;
+  }
+  return G;
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_sh,
@@ -152,11 +199,15 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   SharedState& S = *reinterpret_cast<SharedState*>(smem + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = args.E;
-  const PlanView pv = plan_view(const_cast<int*>(args.plan), E);
-  const int* tp = (MODE == kGateUp) ? pv.tp1 : pv.tp2;
-  const int chunk_max = (MODE == kGateUp) ? kTcChunk : kTcChunkDown;
-  const int total = tp[E + 1];
-  const int R = pv.row0[E];
+  PlanView pv{};
+  int total, R = 0;
+  if (MODE == kRouter) {
+    total = args.ntiles;
+  } else {
+    pv = plan_view(const_cast<int*>(args.plan), E);
+    total = ((MODE == kGateUp) ? pv.tp1 : pv.tp2)[E + 1];
+    R = pv.row0[E];
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -188,33 +239,22 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 #pragma unroll
     for (int s = 0; s < kStages; ++s) armed[s] = -1;
     int aborted = 0;
+    const int plane_rows = (MODE == kDown) ? (int)(args.h_plane / (size_t)args.ldh) : 0;
     for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
-      const Tile tl = decode_tile(pv, tp, E, tile, chunk_max);
-      const bool sh = tl.g == E;
-      const CUtensorMap* ta = sh ? &tm_a_sh : &tm_a;
-      int a_row0, a_row1, nk;
+      const Geom G = tile_geom<MODE>(args, pv, tile);
+      const Tile& tl = G.t;
+      const CUtensorMap* ta = G.shared ? &tm_a_sh : &tm_a;
       if (MODE == kGateUp) {
-        const int Ig = sh ? args.Is : args.I;
-        const int base = sh ? 0 : tl.g * 2 * args.I;
-        a_row0 = base + tl.m * 128;
-        a_row1 = base + Ig + tl.m * 128;
-        nk = args.H / 64;
         for (int j = lane; j < tl.N; j += 32) {
           const int q = j < tl.nvalid ? j : tl.nvalid - 1;  // pad with the last real row
           S.tok[j] = token_of_row(args, tl.p0 + q, R);
         }
         __syncwarp();
-      } else {
-        const int base = sh ? 0 : tl.g * args.H;
-        a_row0 = base + tl.m * 256;
-        a_row1 = a_row0 + 128;
-        nk = (sh ? args.Is : args.I) / 64;
       }
       if (lane == 0) {
-        const int brows = (MODE == kGateUp) ? tl.N : 2 * tl.N;
+        const int brows = (MODE == kDown) ? 2 * tl.N : tl.N;
         const uint32_t bytes = 2 * kATileBytes + (uint32_t)brows * 128u;
-        const int plane_rows = (int)(args.h_plane / (size_t)args.ldh);
-        for (int ks = 0; ks < nk; ++ks, ++it) {
+        for (int ks = 0; ks < G.nk; ++ks, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
           if (!wait_phase(&S.empty[s], ph ^ 1u, S, args.status)) {
@@ -224,19 +264,23 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           ptx::mbar_arrive_expect_tx(&S.full[s], bytes);
           armed[s] = (int)ph;
           uint8_t* st = smem + s * kStageBytes;
-          ptx::tma_load_2d(st, ta, &S.full[s], ks * 64, a_row0);
-          ptx::tma_load_2d(st + kATileBytes, ta, &S.full[s], ks * 64, a_row1);
+          ptx::tma_load_2d(st, ta, &S.full[s], ks * 64, G.a_row0);
+          ptx::tma_load_2d(st + kATileBytes, ta, &S.full[s], ks * 64, G.a_row1);
           uint8_t* b = st + 2 * kATileBytes;
           if (MODE == kGateUp) {
             for (int j = 0; j < tl.N; j += 4)
               ptx::tma_gather4(b + j * 128, &tm_b, &S.full[s], ks * 64, S.tok[j], S.tok[j + 1],
                                S.tok[j + 2], S.tok[j + 3]);
-          } else {
+          } else if (MODE == kDown) {
             for (int j = 0; j < tl.N; j += 16) {
               ptx::tma_load_2d(b + j * 128, &tm_b, &S.full[s], ks * 64, tl.p0 + j);
               ptx::tma_load_2d(b + (tl.N + j) * 128, &tm_b, &S.full[s], ks * 64,
                                plane_rows + tl.p0 + j);
             }
+          } else {
+            const int kx = (ks * 64) % args.H;  // the same x columns for each router piece
+            for (int j = 0; j < tl.N; j += 16)
+              ptx::tma_load_2d(b + j * 128, &tm_b, &S.full[s], kx, tl.p0 + j);
           }
         }
       }
@@ -254,17 +298,15 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       int it = 0, tcount = 0;
       bool aborted = false;
       for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x, ++tcount) {
-        const Tile tl = decode_tile(pv, tp, E, tile, chunk_max);
-        const bool sh = tl.g == E;
-        const int nk = (MODE == kGateUp) ? args.H / 64 : (sh ? args.Is : args.I) / 64;
-        const int nmma = (MODE == kGateUp) ? tl.N : 2 * tl.N;
+        const Geom G = tile_geom<MODE>(args, pv, tile);
+        const int nmma = (MODE == kDown) ? 2 * G.t.N : G.t.N;
         const uint32_t idesc = ptx::idesc_bf16_f32(128, nmma);
         if (!wait_phase(&S.tmem_empty, ((uint32_t)tcount & 1u) ^ 1u, S, args.status)) {
           aborted = true;
           break;
         }
         ptx::tc_fence_after();
-        for (int ks = 0; ks < nk; ++ks, ++it) {
+        for (int ks = 0; ks < G.nk; ++ks, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
           if (!wait_phase(&S.full[s], ph, S, args.status)) {
@@ -300,7 +342,8 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
     int tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
-      const Tile tl = decode_tile(pv, tp, E, tile, chunk_max);
+      const Geom G = tile_geom<MODE>(args, pv, tile);
+      const Tile& tl = G.t;
       const bool ok = wait_phase(&S.tmem_full, (uint32_t)tcount & 1u, S, args.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       ptx::tc_fence_after();
@@ -320,6 +363,22 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
               const size_t at = (size_t)(tl.p0 + c0 + j) * args.ldh + ch;
               args.h[at] = hi;
               args.h[args.h_plane + at] = f32_to_bf16_rn(hv - bf16lo(hi));
+            }
+          }
+        }
+      } else if (MODE == kRouter) {
+        const int e0 = tl.m * 256 + qd * 32 + lane;  // experts e0 and e0 + 128
+        for (int c0 = 0; c0 < tl.nvalid; c0 += 32) {
+          uint32_t l0[32], l1[32];
+          ptx::tmem_ld32(lane_base + c0, l0);
+          ptx::tmem_ld32(lane_base + kAcc1Col + c0, l1);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (c0 + j < tl.nvalid) {
+              float* row = args.logits + (size_t)(tl.p0 + c0 + j) * E;
+              if (e0 < E) row[e0] = __uint_as_float(l0[j]);
+              if (e0 + 128 < E) row[e0 + 128] = __uint_as_float(l1[j]);
             }
           }
         }
@@ -380,6 +439,27 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Router matrix fp32 [E][H] -> bf16 pieces [E][3H] = hi | mid | lo with
+// w = hi + mid + lo exactly (each piece takes the next 8 significant bits), so every
+// product with a bf16 activation is exact and the tensor-core sum is an fp32 dot product.
+__global__ void router_split_kernel(const float* __restrict__ wr, uint16_t* __restrict__ out,
+                                    int E, int H) {
+  const size_t n = (size_t)E * H;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t e = i / H, h = i % H;
+    const float w = wr[i];
+    const uint16_t hi = f32_to_bf16_rn(w);
+    const float r1 = w - bf16lo(hi);
+    const uint16_t mid = f32_to_bf16_rn(r1);
+    const float r2 = r1 - bf16lo(mid);
+    uint16_t* row = out + e * 3 * (size_t)H;
+    row[h] = hi;
+    row[H + h] = mid;
+    row[2 * H + h] = f32_to_bf16_rn(r2);
   }
 }
 
@@ -451,6 +531,45 @@ TcArgs base_args(const moe_shape& s, const Layout& L, char* ws) {
 }
 
 }  // namespace
+
+bool tc_router_supported(const moe_shape& s) {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return false;
+  return major == 10 && encode_fn() != nullptr && s.H % 64 == 0;
+}
+
+cudaError_t launch_tc_router(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
+                             const float* wr, float* logits, cudaStream_t st) {
+  uint16_t* split = reinterpret_cast<uint16_t*>(ws + L.wr_split);
+  {
+    LaunchScope scope(MOE_K_OTHER, st);
+    const size_t n = (size_t)s.E * s.H;
+    const int blocks = (int)std::min<size_t>((n + 255) / 256, (size_t)sm_count() * 8);
+    router_split_kernel<<<blocks, 256, 0, st>>>(wr, split, s.E, s.H);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap a, b;
+  if (!make_map(&a, split, 3ull * s.H, (uint64_t)s.E, 64, 128) ||
+      !make_map(&b, x, s.H, (uint64_t)s.T, 64, 16))
+    return cudaErrorInvalidValue;
+  TcArgs args = base_args(s, L, ws);
+  args.logits = logits;
+  args.ntiles = ((s.E + 255) / 256) * ((s.T + 255) / 256);
+  LaunchScope scope(MOE_K_ROUTER_LOGITS, st);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(tc_grouped_kernel<kRouter>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int grid = std::min(args.ntiles, sm_count());
+  tc_grouped_kernel<kRouter><<<grid, kThreads, kSmemBytes, st>>>(a, a, b, args);
+  return cudaGetLastError();
+}
 
 bool tc_supported(const moe_shape& s) {
   if (s.I % 128 || s.Is % 128 || s.H % 256) return false;
