@@ -135,6 +135,25 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_ids, int32_t*
                        void* stream);
 
 /*
+ * moe_permute without a workspace, for callers that cannot allocate device memory: code
+ * that runs where an allocation would block or is not allowed (inside a real-time serving
+ * loop that must not enter the allocator, a plugin host that hands a custom op only its
+ * input and output buffers, a process whose memory pool is already fully reserved).
+ * The pages have no counterpart; it computes exactly what moe_permute computes (same
+ * offsets, sorted_token, assign_row), with the same argument meaning and layout.
+ * Its scratch is a fixed 640 KB array inside this library, held on every GPU that loads
+ * the library until the process exits; it allocates nothing and calls no allocating
+ * routine. Limit: ceil(T/256) * E <= 16384 (for example T <= 8192 with E = 512); larger
+ * shapes return MOE_ERR_UNSUPPORTED (use moe_permute with a workspace). The first call on
+ * a device looks up the array's device address; make that first call before capturing a
+ * stream into a CUDA graph. All calls share the one array: calls that overlap on the GPU
+ * (different streams, or several host threads) race and give wrong results. An id outside
+ * [0, E) is skipped; offsets[E] then falls short of T*k.
+ */
+moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_ids, int32_t* offsets,
+                               int32_t* sorted_token, int32_t* assign_row, void* stream);
+
+/*
  * Stage 4: "Grouped expert GEMMs" with the layer's expert formula
  * expert(x) = W_down(SiLU(W_gate x) * W_up x). Unweighted per-assignment outputs:
  *   y[p,:]        = expert_{e(p)}(x[sorted_token[p],:])   fp32 [T*k][H] (packed order)

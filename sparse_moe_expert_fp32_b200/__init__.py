@@ -68,6 +68,7 @@ _SIGS = {
     "moe_workspace_init": ([_vp, _sz, _vp], ctypes.c_int),
     "moe_router_topk": ([_SP, _vp, _WP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_permute": ([_SP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_permute_noalloc": ([_SP, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moe_grouped_swiglu": ([_SP, _vp, _vp, _vp, _WP, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_unpermute_combine": ([_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moe_layer_forward": ([_SP, _vp, _WP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
@@ -175,6 +176,13 @@ def moe_router_topk(shape, x, weights, topk_ids, topk_w, shared_gate, gap, ws, s
 def moe_permute(shape, topk_ids, offsets, sorted_token, assign_row, ws, stream=None):
     _check(_lib.moe_permute(ctypes.byref(shape), _ptr(topk_ids), _ptr(offsets), _ptr(sorted_token),
                             _ptr(assign_row), _ptr(ws), _nbytes(ws), _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(shape, topk_ids, offsets, sorted_token, assign_row, stream=None):
+    """moe_permute for callers that cannot allocate: no workspace, fixed internal scratch."""
+    _check(_lib.moe_permute_noalloc(ctypes.byref(shape), _ptr(topk_ids), _ptr(offsets),
+                                    _ptr(sorted_token), _ptr(assign_row), _stream(stream)),
+           "moe_permute_noalloc")
 
 
 def moe_grouped_swiglu(shape, x, sorted_token, offsets, weights, y, y_shared, ws, stream=None):

@@ -13,6 +13,8 @@
 //                           the same mask -- token-ascending inside each expert, and the
 //                           same on every run.
 // An expert id outside [0, E) is skipped and raises the bounds flag in the status word.
+#include <mutex>
+
 #include "device_common.cuh"
 #include "moe_internal.h"
 
@@ -238,4 +240,102 @@ cudaError_t launch_plan_from_offsets(const moe_shape& s, const Layout& L, char* 
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- no-allocation dispatch
+//
+// moe_permute_noalloc: the dispatch above for callers that cannot allocate device memory
+// (no workspace argument). Its scratch -- status word, per-block token masks and bases,
+// GEMM plan -- lives in one file-scope device array that every GPU loading this library
+// holds until the process exits. In host code `g_noalloc_scratch` is only a host-side
+// stand-in for the symbol; its device address is looked up with cudaGetSymbolAddress,
+// once per device, with that device current (the first call on a device does it).
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 640u * 1024u;
+constexpr long long kNoAllocMaxBlockExperts = 16384;  // ceil(T/256) * E
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices];
+
+cudaError_t noalloc_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+
+struct NoAllocLayout {
+  size_t status, blk_mask, blk_base, plan, total;
+  int nblk;
+};
+
+NoAllocLayout noalloc_layout(const moe_shape& s) {
+  NoAllocLayout L{};
+  L.nblk = (s.T + kPermBlock - 1) / kPermBlock;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  L.status = take(256);
+  L.blk_mask = take((size_t)L.nblk * s.E * 8 * sizeof(uint32_t));
+  L.blk_base = take((size_t)L.nblk * s.E * sizeof(int32_t));
+  L.plan = take(plan_ints(s.E) * sizeof(int32_t));
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
 }  // namespace moe
+
+extern "C" moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_ids,
+                                          int32_t* offsets, int32_t* sorted_token,
+                                          int32_t* assign_row, void* stream) {
+  using namespace moe;
+  if (!shape) return MOE_ERR_INVALID_ARG;
+  const moe_shape& s = *shape;
+  if (s.T < 0 || s.E <= 0 || s.k <= 0 || s.H <= 0 || s.I <= 0 || s.Is <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (s.E > kMaxE || s.k > kMaxK || s.k > s.E || s.H % 64 || s.I % 64 || s.Is % 64)
+    return MOE_ERR_UNSUPPORTED;
+  auto a16 = [](const void* p) { return p && ((uintptr_t)p & 15u) == 0; };
+  if (!a16(topk_ids) || !a16(offsets) || !a16(sorted_token) || !a16(assign_row))
+    return MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  const NoAllocLayout L = noalloc_layout(s);
+  if ((long long)L.nblk * s.E > kNoAllocMaxBlockExperts || L.total > kNoAllocScratchBytes)
+    return MOE_ERR_UNSUPPORTED;  // beyond the fixed scratch: use moe_permute with a workspace
+  void* base = nullptr;
+  if (noalloc_scratch_address(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  char* ws = static_cast<char*>(base);
+  cudaStream_t st = (cudaStream_t)stream;
+  // the array keeps the previous call's contents: clear the status word; the masks are
+  // rebuilt in shared memory and the bases and plan are fully rewritten by every call
+  if (cudaMemsetAsync(ws + L.status, 0, 256, st) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  uint32_t* blk_mask = reinterpret_cast<uint32_t*>(ws + L.blk_mask);
+  int32_t* blk_base = reinterpret_cast<int32_t*>(ws + L.blk_base);
+  const size_t smem = (size_t)s.E * 8 * sizeof(uint32_t);
+  dispatch_mask_kernel<<<L.nblk, kPermBlock, smem, st>>>(topk_ids, s.T, s.E, s.k, blk_mask,
+                                                        blk_base, status);
+  dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(blk_base, L.nblk, s.T, s.E, s.k, s.H, s.I,
+                                                   s.Is, blk_base, offsets,
+                                                   reinterpret_cast<int*>(ws + L.plan));
+  dispatch_scatter_kernel<<<L.nblk, kPermBlock, 0, st>>>(topk_ids, nullptr, s.T, s.E, s.k,
+                                                         blk_mask, blk_base, sorted_token,
+                                                         nullptr, assign_row);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
