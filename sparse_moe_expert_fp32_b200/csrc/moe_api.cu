@@ -25,7 +25,7 @@ Layout layout(const moe_shape& s) {
     return at;
   };
   L.status = take(64 * sizeof(uint32_t));
-  L.logits = take(T * E * sizeof(float));
+  L.logits = take((T < 512 ? 4 : 1) * T * E * sizeof(float));
   L.wr_split = take(E * 3 * H * sizeof(uint16_t));
   L.ids = take(R * sizeof(int32_t));
   L.w = take(R * sizeof(float));
@@ -38,6 +38,7 @@ Layout layout(const moe_shape& s) {
   L.sorted_w = take(R * sizeof(float));
   L.assign_row = take(R * sizeof(int32_t));
   L.plan = take(plan_ints(s.E) * sizeof(int32_t));
+  L.xs = take(R * H * sizeof(uint16_t));
   L.h_plane = (R + T) * (size_t)L.ldh;
   L.h = take(2 * L.h_plane * sizeof(uint16_t));
   L.total = o;
@@ -199,7 +200,8 @@ moe_status moe_router_topk(const moe_shape* shape, const void* x, const moe_weig
   float* logits = reinterpret_cast<float*>(w + L.logits);
   MOE_CUDA(launch_router_logits(s, L, w, static_cast<const uint16_t*>(x), weights->w_router,
                                 logits, st));
-  MOE_CUDA(launch_router_topk(s, logits, weights->router_bias, static_cast<const uint16_t*>(x),
+  MOE_CUDA(launch_router_topk(s, logits, weights->w_router, weights->router_bias,
+                              static_cast<const uint16_t*>(x),
                               static_cast<const uint16_t*>(weights->w_shared_gate), topk_ids,
                               topk_w, shared_gate, gap, nullptr, st));
   return MOE_OK;
@@ -279,7 +281,7 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, const moe_we
   float* sorted_w = reinterpret_cast<float*>(w + L.sorted_w);
 
   MOE_CUDA(launch_router_logits(s, L, w, xb, weights->w_router, logits, st));
-  MOE_CUDA(launch_router_topk(s, logits, weights->router_bias, xb,
+  MOE_CUDA(launch_router_topk(s, logits, weights->w_router, weights->router_bias, xb,
                               static_cast<const uint16_t*>(weights->w_shared_gate), ids, tw, sg,
                               gap, out /* rows zeroed here, accumulated by the down GEMM */, st));
   MOE_CUDA(launch_permute(s, L, w, ids, tw, reinterpret_cast<int32_t*>(w + L.offsets),

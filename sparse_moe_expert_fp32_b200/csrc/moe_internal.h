@@ -13,7 +13,7 @@ namespace moe {
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 32;
 constexpr int kPermBlock = 256;  // tokens per dispatch block (one bit per token in a mask)
-constexpr int kTcChunk = 256;    // max tokens (MMA N) per tensor-core tile
+constexpr int kTcChunk = 128;    // max tokens (MMA N) per tensor-core tile
 constexpr uint32_t kFlagBounds = 1u;
 constexpr uint32_t kFlagTimeout = 2u;
 
@@ -22,7 +22,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Byte offsets of the workspace regions (all 256-byte aligned).
 struct Layout {
   size_t status;        // uint32 [64]: [0] = error flags, [1..] = diagnostics
-  size_t logits;        // fp32 [T][E]
+  size_t logits;        // fp32 [4][T][E] partial router logits for T < 512, else [T][E]
   size_t wr_split;      // bf16 [E][3H]: router matrix as hi|mid|lo bf16 pieces (tensor-core router)
   size_t ids;           // int32 [T][k]
   size_t w;             // fp32 [T][k]
@@ -35,6 +35,7 @@ struct Layout {
   size_t sorted_w;      // fp32 [T*k]: routing weight of each packed row
   size_t assign_row;    // int32 [T*k]
   size_t plan;          // int32 plan arrays (see PlanView)
+  size_t xs;            // bf16 [T*k][H]: token rows in dispatch order (tensor-core gate|up)
   size_t h;             // bf16 [2][T*k + T][ldh]: SwiGLU intermediate as a hi|lo pair of planes
                         // (h = hi + lo), routed rows then shared rows
   size_t h_plane;       // elements per plane: (T*k + T) * ldh
@@ -69,9 +70,8 @@ __host__ __device__ inline PlanView plan_view(void* base, int E) {
 }
 
 // Tensor-core tiling of a group with n rows into ceil(n / max) token chunks of nearly equal
-// size (multiples of 16 rows): max 256 rows for the gate|up GEMM, 128 for the down GEMM
-// (whose B operand holds the hi and lo rows of each token).
-constexpr int kTcChunkDown = 128;
+// size (multiples of 16 rows), max 128 rows for both grouped GEMMs.
+constexpr int kTcChunkDown = kTcChunk;
 __host__ __device__ inline int tc_nchunks(int n, int max_rows) {
   return (n + max_rows - 1) / max_rows;
 }
@@ -89,13 +89,14 @@ struct LaunchScope {
 // ---------------------------------------------------------------- kernel launches
 // Every launcher enqueues on `st` and returns cudaGetLastError().
 
-cudaError_t launch_router_logits_stream(const moe_shape& s, const uint16_t* x, const float* wr,
-                                        float* logits, cudaStream_t st);
-// router logits by the best available kernel for the shape (uses the workspace)
+// Router logits by the best kernel for the shape (uses the workspace). Small batches leave
+// router_slices(s) partial sums [slices][T][E] that launch_router_topk adds up.
 cudaError_t launch_router_logits(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                                  const float* wr, float* logits, cudaStream_t st);
-cudaError_t launch_router_topk(const moe_shape& s, const float* logits, const float* bias,
-                               const uint16_t* x, const uint16_t* wsg, int32_t* ids, float* w,
+int router_slices(const moe_shape& s);
+cudaError_t launch_router_topk(const moe_shape& s, const float* logits, const float* wr,
+                               const float* bias, const uint16_t* x, const uint16_t* wsg,
+                               int32_t* ids, float* w,
                                float* sgate, float* gap, float* out_zero, cudaStream_t st);
 cudaError_t launch_permute(const moe_shape& s, const Layout& L, char* ws, const int32_t* ids,
                            const float* topk_w, int32_t* offsets, int32_t* sorted_token,

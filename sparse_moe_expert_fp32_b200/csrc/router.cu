@@ -3,9 +3,9 @@
 // normalises the selected router probabilities; the shared expert has its own sigmoid
 // output gate).
 //
-//   router_logits_stream_kernel : logits = x . Wr^T on CUDA cores, fp32 accumulation
-//                                 (small batches; larger ones use the tensor-core router
-//                                 in tc_gemm.cu).
+//   router_logits_small_kernel  : logits = x . Wr^T on CUDA cores for small batches, as
+//                                 four partial sums over hidden-dimension slices; larger
+//                                 batches use the tensor-core router in tc_gemm.cu.
 //   router_topk_kernel          : one warp per token: top-k with lowest-index ties,
 //                                 renormalised softmax weights, 10th/11th gap,
 //                                 shared-expert gate sigmoid(w_shared . x).
@@ -18,90 +18,99 @@
 namespace moe {
 namespace {
 
-constexpr int kRouterWarps = 8;
-constexpr int kRowsPerWarp = 8;  // router rows (experts) per warp
-constexpr int kTokPerWarp = 4;   // tokens per warp
+// Small batches (T < 512): partial logits over kSplits slices of the hidden dimension,
+// part[s][t][e] = sum_{h in slice s} x[t][h] * wr[e][h], fp32 FMAs in h order. A CTA
+// computes 16 experts x 64 tokens of one slice: x and wr chunks are staged in shared
+// memory (x transposed so that a warp's 32 tokens read consecutive words), each thread
+// accumulates 4 experts x 1 token. The top-k kernel adds the slices in order s = 0..3, so
+// the logits are the same on every run. Grid (ceil(E/16), kSplits, ceil(T/64)) fills the
+// GPU at decode sizes (128 CTAs at E = 512, T = 64) and reads wr once.
+constexpr int kSplits = 4;
+constexpr int kSmallTok = 64;
+constexpr int kSmallExp = 16;
+constexpr int kSmallKc = 128;
 
-// logits[t][e] = sum_h x[t][h] * wr[e][h]. A warp computes 8 experts x 4 tokens; lanes
-// stride over h in chunks of 4 elements; the 32 partial sums are combined with one
-// transpose-reduction. Grid: (ceil(E/64), ceil(T/4)).
-__global__ void __launch_bounds__(kRouterWarps * 32)
-router_logits_stream_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
-                            float* __restrict__ logits, int T, int H, int E) {
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int e0 = (blockIdx.x * kRouterWarps + warp) * kRowsPerWarp;
-  const int t0 = blockIdx.y * kTokPerWarp;
-  if (e0 >= E) return;
+__global__ void __launch_bounds__(256)
+router_logits_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
+                           float* __restrict__ part, int T, int H, int E, int nslices) {
+  __shared__ float xs[kSmallKc][kSmallTok];
+  __shared__ float4 wsm[kSmallKc][kSmallExp / 4];
+  const int e0 = blockIdx.x * kSmallExp;
+  const int t0 = blockIdx.z * kSmallTok;
+  const int slice = H / nslices;  // a multiple of 16 (H is a multiple of 64)
+  const int kbeg = blockIdx.y * slice, kend = kbeg + slice;
+  const int tid = threadIdx.x;
+  const int tok = tid & (kSmallTok - 1), eg = tid >> 6;  // 4 expert groups of 4
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
 
-  float acc[32];
+  for (int k0 = kbeg; k0 < kend; k0 += kSmallKc) {
+    const int kn = min(kSmallKc, kend - k0);  // multiple of 16
+    const int x8 = kn / 8;
+    for (int i = tid; i < kSmallTok * x8; i += blockDim.x) {
+      const int r = i % kSmallTok, c = i / kSmallTok;  // consecutive threads: consecutive tokens
+      float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (t0 + r < T) unpack8(ld_v4(x + (size_t)(t0 + r) * H + k0 + 8 * c), f);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-
-  const int nchunk = H / 4;
-  for (int c = lane; c < nchunk; c += 32) {
-    float xv[kTokPerWarp][4];
-#pragma unroll
-    for (int q = 0; q < kTokPerWarp; ++q) {
-      const int t = t0 + q;
-      if (t < T) {
-        uint2 u = __ldg(reinterpret_cast<const uint2*>(x + (size_t)t * H + 4 * c));
-        xv[q][0] = bf16lo(u.x); xv[q][1] = bf16hi(u.x);
-        xv[q][2] = bf16lo(u.y); xv[q][3] = bf16hi(u.y);
-      } else {
-        xv[q][0] = xv[q][1] = xv[q][2] = xv[q][3] = 0.f;
-      }
+      for (int j = 0; j < 8; ++j) xs[8 * c + j][r] = f[j];
     }
+    const int w4 = kn / 4;
+    for (int i = tid; i < kSmallExp * w4; i += blockDim.x) {
+      const int e = i % kSmallExp, c = i / kSmallExp;  // consecutive threads: consecutive experts
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e0 + e < E) v = __ldg(reinterpret_cast<const float4*>(wr + (size_t)(e0 + e) * H + k0) + c);
+      float* col = reinterpret_cast<float*>(&wsm[0][0]) + e;
+      col[(4 * c + 0) * kSmallExp] = v.x;
+      col[(4 * c + 1) * kSmallExp] = v.y;
+      col[(4 * c + 2) * kSmallExp] = v.z;
+      col[(4 * c + 3) * kSmallExp] = v.w;
+    }
+    __syncthreads();
+    for (int kk = 0; kk < kn; ++kk) {
+      const float xv = xs[kk][tok];
+      const float4 w = wsm[kk][eg];
+      acc[0] = fmaf(xv, w.x, acc[0]);
+      acc[1] = fmaf(xv, w.y, acc[1]);
+      acc[2] = fmaf(xv, w.z, acc[2]);
+      acc[3] = fmaf(xv, w.w, acc[3]);
+    }
+    __syncthreads();
+  }
+  const int t = t0 + tok;
+  if (t < T) {
+    float* row = part + ((size_t)blockIdx.y * T + t) * E;
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-      const int e = e0 + r;
-      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E) w = __ldg(reinterpret_cast<const float4*>(wr + (size_t)e * H + 4 * c));
-#pragma unroll
-      for (int q = 0; q < kTokPerWarp; ++q) {
-        float a = acc[r * 4 + q];
-        a = fmaf(w.x, xv[q][0], a);
-        a = fmaf(w.y, xv[q][1], a);
-        a = fmaf(w.z, xv[q][2], a);
-        a = fmaf(w.w, xv[q][3], a);
-        acc[r * 4 + q] = a;
-      }
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + eg * 4 + j;
+      if (e < E) row[e] = acc[j];
     }
   }
-  const float s = warp_transpose_sum32(acc, lane);
-  const int e = e0 + lane / 4;
-  const int t = t0 + lane % 4;
-  if (e < E && t < T) logits[(size_t)t * E + e] = s;
 }
 
-// One warp per token. Lane l holds logits of experts l, l+32, ...; VPL = values per lane.
-template <int VPL>
-__global__ void __launch_bounds__(256)
-router_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
-                   const uint16_t* __restrict__ x, const uint16_t* __restrict__ wsg, int T, int H,
-                   int E, int k, int32_t* __restrict__ ids, float* __restrict__ w,
-                   float* __restrict__ sgate, float* __restrict__ gap,
-                   float* __restrict__ out_zero) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-
-  float v[VPL];
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int e = lane + 32 * i;
-    float l = -FLT_MAX;
-    if (e < E) {
-      l = logits[(size_t)t * E + e];
-      if (bias) l += bias[e];
-    }
-    v[i] = l;
+// x[t] . wr[e] in fp32 FMAs (lane-strided over h, then a warp sum); every lane gets it.
+__device__ __forceinline__ float exact_logit(const uint16_t* xr, const float* wrow, int H, int lane) {
+  float acc = 0.f;
+  for (int c = lane; c < H / 8; c += 32) {
+    float xf[8];
+    unpack8(ld_v4(xr + 8 * c), xf);
+    const float4 a = __ldg(reinterpret_cast<const float4*>(wrow + 8 * c));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(wrow + 8 * c) + 1);
+    acc = fmaf(a.x, xf[0], acc); acc = fmaf(a.y, xf[1], acc);
+    acc = fmaf(a.z, xf[2], acc); acc = fmaf(a.w, xf[3], acc);
+    acc = fmaf(b.x, xf[4], acc); acc = fmaf(b.y, xf[5], acc);
+    acc = fmaf(b.z, xf[6], acc); acc = fmaf(b.w, xf[7], acc);
   }
+  return warp_sum(acc);
+}
 
+// Top-(k+1) by (value desc, index asc) over the lane-held values; lanes r < k receive the
+// r-th (id, value), every lane the (k+1)-th value.
+template <int VPL>
+__device__ __forceinline__ void select_topk(const float (&v)[VPL], int E, int k, int lane,
+                                            int& my_id, float& my_val, float& next_val) {
   uint32_t taken = 0;
-  int my_id = 0;
-  float my_val = 0.f;
-  float next_val = -FLT_MAX;  // (k+1)-th largest
+  my_id = 0;
+  my_val = 0.f;
+  next_val = -FLT_MAX;
   const int rounds = (k < E) ? k + 1 : k;
   for (int r = 0; r < rounds; ++r) {
     float bv = -FLT_MAX;
@@ -131,6 +140,62 @@ router_topk_kernel(const float* __restrict__ logits, const float* __restrict__ b
       }
     } else {
       next_val = bv;
+    }
+  }
+}
+
+// One warp per token. Lane l holds logits of experts l, l+32, ...; VPL = values per lane.
+// `logits` holds `nslices` partial sums [nslices][T][E], added in slice order.
+// With `wr` set (logits from the tensor-core router, whose accumulation is not exact fp32),
+// a token whose k-th / (k+1)-th gap is below `band` has every expert within `band` of the
+// k-th logit recomputed as an exact fp32 dot product, and the selection is redone on those
+// values: the choice then matches fp32 arithmetic except at true near-ties.
+template <int VPL>
+__global__ void __launch_bounds__(256)
+router_topk_kernel(const float* __restrict__ logits, int nslices, const float* __restrict__ bias,
+                   const uint16_t* __restrict__ x, const uint16_t* __restrict__ wsg,
+                   const float* __restrict__ wr, float band, int T, int H, int E, int k,
+                   int32_t* __restrict__ ids, float* __restrict__ w, float* __restrict__ sgate,
+                   float* __restrict__ gap, float* __restrict__ out_zero) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+
+  float v[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane + 32 * i;
+    float l = -FLT_MAX;
+    if (e < E) {
+      l = logits[(size_t)t * E + e];
+      for (int sl = 1; sl < nslices; ++sl) l += logits[((size_t)sl * T + t) * E + e];
+      if (bias) l += bias[e];
+    }
+    v[i] = l;
+  }
+
+  int my_id;
+  float my_val, next_val;
+  select_topk<VPL>(v, E, k, lane, my_id, my_val, next_val);
+  if (wr && k < E) {
+    const float kth = __shfl_sync(0xffffffffu, my_val, k - 1);
+    if (kth - next_val < band) {
+      const float lo = kth - band;
+      const uint16_t* xr = x + (size_t)t * H;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int e_l = lane + 32 * i;
+        uint32_t m = __ballot_sync(0xffffffffu, e_l < E && v[i] >= lo);
+        while (m) {
+          const int src = __ffs(m) - 1;
+          m &= m - 1;
+          const int e = src + 32 * i;
+          float l = exact_logit(xr, wr + (size_t)e * H, H, lane);
+          if (bias) l += bias[e];
+          if (lane == src) v[i] = l;
+        }
+      }
+      select_topk<VPL>(v, E, k, lane, my_id, my_val, next_val);
     }
   }
 
@@ -166,36 +231,40 @@ router_topk_kernel(const float* __restrict__ logits, const float* __restrict__ b
 
 }  // namespace
 
-cudaError_t launch_router_logits_stream(const moe_shape& s, const uint16_t* x, const float* wr,
-                                        float* logits, cudaStream_t st) {
-  LaunchScope scope(MOE_K_ROUTER_LOGITS, st);
-  dim3 grid((s.E + kRouterWarps * kRowsPerWarp - 1) / (kRouterWarps * kRowsPerWarp),
-            (s.T + kTokPerWarp - 1) / kTokPerWarp);
-  router_logits_stream_kernel<<<grid, kRouterWarps * 32, 0, st>>>(x, wr, logits, s.T, s.H, s.E);
-  return cudaGetLastError();
-}
-
 // Token count from which the tensor-core router (a GEMM over the exact three-piece split
 // of the router matrix) replaces the CUDA-core one.
 constexpr int kTcRouterMinTokens = 512;
+// Half-width of the band of tensor-core logits that is recomputed exactly around the k-th
+// (several times the largest deviation of those logits from fp32 dot products).
+constexpr float kRefineBand = 4e-3f;
+
+int router_slices(const moe_shape& s) { return s.T < kTcRouterMinTokens ? kSplits : 1; }
 
 cudaError_t launch_router_logits(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                                  const float* wr, float* logits, cudaStream_t st) {
-  if (s.T >= kTcRouterMinTokens && tc_router_supported(s))
-    return launch_tc_router(s, L, ws, x, wr, logits, st);
-  return launch_router_logits_stream(s, x, wr, logits, st);
+  const int nslices = router_slices(s);
+  const bool tc_logits = nslices == 1 && tc_router_supported(s);
+  if (nslices == 1 && tc_router_supported(s)) return launch_tc_router(s, L, ws, x, wr, logits, st);
+  LaunchScope scope(MOE_K_ROUTER_LOGITS, st);
+  dim3 grid((s.E + kSmallExp - 1) / kSmallExp, nslices, (s.T + kSmallTok - 1) / kSmallTok);
+  router_logits_small_kernel<<<grid, 256, 0, st>>>(x, wr, logits, s.T, s.H, s.E, nslices);
+  return cudaGetLastError();
 }
 
-cudaError_t launch_router_topk(const moe_shape& s, const float* logits, const float* bias,
-                               const uint16_t* x, const uint16_t* wsg, int32_t* ids, float* w,
+cudaError_t launch_router_topk(const moe_shape& s, const float* logits, const float* wr,
+                               const float* bias, const uint16_t* x, const uint16_t* wsg,
+                               int32_t* ids, float* w,
                                float* sgate, float* gap, float* out_zero, cudaStream_t st) {
   LaunchScope scope(MOE_K_ROUTER_TOPK, st);
+  const int nslices = router_slices(s);
+  const bool tc_logits = nslices == 1 && tc_router_supported(s);
   const int warps = 8;
   dim3 grid((s.T + warps - 1) / warps);
   const int vpl = (s.E + 31) / 32;
 #define MOE_TOPK_CASE(N)                                                                     \
-  router_topk_kernel<N><<<grid, warps * 32, 0, st>>>(logits, bias, x, wsg, s.T, s.H, s.E, s.k, \
-                                                     ids, w, sgate, gap, out_zero)
+  router_topk_kernel<N><<<grid, warps * 32, 0, st>>>(logits, nslices, bias, x, wsg,             \
+                                                     tc_logits ? wr : nullptr, kRefineBand, s.T, s.H, \
+                                                     s.E, s.k, ids, w, sgate, gap, out_zero)
   if (vpl <= 1) MOE_TOPK_CASE(1);
   else if (vpl <= 2) MOE_TOPK_CASE(2);
   else if (vpl <= 4) MOE_TOPK_CASE(4);

@@ -1,27 +1,31 @@
 // tc_gemm.cu -- stage 4, "Grouped expert GEMMs" (Qwen3.8-Flash-Next architecture study,
-// MoE pipeline diagram; expert(x) = W_down(SiLU(W_gate x) * W_up x)) on the 5th-generation
-// tensor cores: TMA-fed shared-memory ring, tcgen05.mma with fp32 accumulators in tensor
-// memory, and fused epilogues.
+// MoE pipeline diagram; expert(x) = W_down(SiLU(W_gate x) * W_up x)), and the router GEMM
+// of stage 1, on the 5th-generation tensor cores: TMA-fed shared-memory ring,
+// tcgen05.mma with fp32 accumulators in tensor memory, fused epilogues.
 //
-// Orientation ("swap AB"): expert weight rows are the MMA's M side (128 rows per
-// accumulator), the tokens of one expert are the N side (16..256 per tile), K is the
-// hidden (gate|up) or intermediate (down) dimension. Every weight byte is read from HBM
-// once per token chunk; token rows come from L2.
+// Orientation ("swap AB"): weight rows are the MMA's M side (two 128-row accumulators per
+// tile = 256 weight rows sharing one token tile), the tokens of one expert are the N side
+// (multiples of 16, at most 128 per tile), K is the hidden (gate|up, router) or
+// intermediate (down) dimension. Every weight byte comes from HBM once per token chunk;
+// the chunks of one weight tile are neighbouring tiles, so a second chunk reads it from L2.
 //
-//   gate|up kernel: per tile, gate rows [c, c+128) and up rows [I+c, I+c+128) of one expert
-//     against up to 256 of its tokens, gathered from x by TMA (tile::gather4) through the
-//     dispatch order. Two accumulators (gate, up) share the token tile. Epilogue:
-//     h = SiLU(gate) * up, stored as the bf16 pair hi = bf16(h), lo = bf16(h - hi).
-//   down kernel: per tile, 256 output rows (two accumulators) of one expert's W_down
-//     against up to 128 of its packed rows; the token tile holds the hi rows followed by
-//     the lo rows, so one MMA with N' = 2N produces W h_hi and W h_lo side by side and the
-//     epilogue adds them. Epilogue: y rows (staged path) or routing-weight-scaled fp32
-//     atomic adds into out[token] ("Weighted combine + gated shared expert").
+//   gate|up: gate rows [c, c+128) and up rows [I+c, I+c+128) of one expert against its
+//     token rows, copied beforehand in dispatch order (gather_rows_kernel) so that a token
+//     tile is a few plain 2-D TMA boxes. Epilogue: h = SiLU(gate) * up stored as the bf16
+//     pair hi = bf16(h), lo = bf16(h - hi).
+//   down: 256 rows of one expert's W_down against its packed rows; per K step two MMAs add
+//     W h_hi and W h_lo into the same accumulators. Epilogue: y rows (staged path) or
+//     routing-weight-scaled fp32 atomic adds into out[token] ("Weighted combine + gated
+//     shared expert").
+//   router: 256 experts x 128 tokens of logits = x . (hi + mid + lo)^T, K = 3H over the
+//     exact bf16 split of the fp32 router matrix.
 //
 // Roles in a 192-thread CTA (one CTA per SM, persistent over the tile list):
-//   warp 0      TMA producer (lane 0 issues), kStages-deep ring of 64 KB stages;
-//   warp 1      TMEM owner (512 columns) and MMA issuer (lane 0);
-//   warps 2..5  epilogue, warp w reads TMEM lanes 32*(w%4) .. +31.
+//   warp 0      TMA producer (lane 0 issues) over a ring of kStages stages;
+//   warp 1      TMEM owner (all 512 columns = two accumulator buffers of 2 x 128 columns)
+//               and MMA issuer (lane 0);
+//   warps 2..5  epilogue, warp w reads TMEM lanes 32*(w%4) .. +31; while it drains one
+//               buffer the MMAs of the next tile fill the other.
 // Every mbarrier wait is bounded (2 s); on expiry the kernel records the timeout flag,
 // lets every role leave its loop, drains its own copies and MMAs and frees TMEM.
 #include <cuda.h>
@@ -37,30 +41,42 @@
 namespace moe {
 namespace {
 
-constexpr int kStages = 3;
 constexpr int kThreads = 192;
-constexpr uint32_t kATileBytes = 128 * 128;      // 128 rows x 64 bf16
-constexpr uint32_t kBTileMaxBytes = 256 * 128;   // 256 rows x 64 bf16
-constexpr uint32_t kStageBytes = 2 * kATileBytes + kBTileMaxBytes;
+constexpr uint32_t kATileBytes = 128 * 128;   // 128 rows x 64 bf16
+constexpr uint32_t kBTileBytes = 128 * 128;   // up to 128 token rows x 64 bf16
+constexpr int kBoxRows = 16;                  // rows per TMA box of a token tile
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAcc1Col = 256;  // column of the second accumulator
+constexpr uint32_t kBufCols = 256;  // one accumulator buffer: two 128-column accumulators
+constexpr int kMaxTile = 128;       // tokens per tile (MMA N)
 
 enum Mode { kGateUp = 0, kDown = 1, kRouter = 2 };
 
+// Stage = two A tiles + one (gate|up, router) or two (down: hi, lo) token tiles.
+template <int MODE>
+struct Cfg {
+  static constexpr int kBTiles = (MODE == kDown) ? 2 : 1;
+  static constexpr uint32_t kStageBytes = 2 * kATileBytes + kBTiles * kBTileBytes;
+  static constexpr int kStages = (MODE == kDown) ? 3 : 4;
+};
+
 struct SharedState {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t tmem_full;
-  uint64_t tmem_empty;
+  uint64_t full[4];
+  uint64_t empty[4];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort;
-  int tok[256];
+  int tp[kMaxE + 2];    // tile prefix of the grouped GEMM (copied from the plan)
+  int row0[kMaxE + 2];  // first packed row of each group (copied from the plan)
 };
 
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(SharedState);
+template <int MODE>
+constexpr size_t smem_bytes() {
+  return 1024 + (size_t)Cfg<MODE>::kStages * Cfg<MODE>::kStageBytes + sizeof(SharedState);
+}
 
 struct TcArgs {
   const int* plan;
@@ -83,10 +99,8 @@ struct Tile {
 };
 
 // Tile -> (group, M tile, packed rows). Groups own consecutive tile ranges
-// [tp[g], tp[g+1]); inside a group the token chunks of one M tile are adjacent, so the
-// second chunk's weight tile is read from L2.
-__device__ __forceinline__ Tile decode_tile(const PlanView& pv, const int* tp, int E, int tile,
-                                            int chunk_max) {
+// [tp[g], tp[g+1]); inside a group the token chunks of one M tile are adjacent.
+__device__ __forceinline__ Tile decode_tile(const int* row0, const int* tp, int E, int tile) {
   int lo = 0, hi = E + 1;  // tp[lo] <= tile < tp[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -95,8 +109,8 @@ __device__ __forceinline__ Tile decode_tile(const PlanView& pv, const int* tp, i
   }
   Tile t;
   t.g = lo;
-  const int n = pv.row0[lo + 1] - pv.row0[lo];
-  const int nch = (n + chunk_max - 1) / chunk_max;
+  const int n = row0[lo + 1] - row0[lo];
+  const int nch = (n + kMaxTile - 1) / kMaxTile;
   const int cs = (((n + nch - 1) / nch) + 15) & ~15;
   const int local = tile - tp[lo];
   t.m = local / nch;
@@ -104,7 +118,7 @@ __device__ __forceinline__ Tile decode_tile(const PlanView& pv, const int* tp, i
   const int start = c * cs;
   t.nvalid = min(cs, n - start);
   t.N = (t.nvalid + 15) & ~15;
-  t.p0 = pv.row0[lo] + start;
+  t.p0 = row0[lo] + start;
   return t;
 }
 
@@ -149,41 +163,44 @@ __device__ __forceinline__ int token_of_row(const TcArgs& a, int p, int R) {
 struct Geom {
   Tile t;
   int a_row0, a_row1;  // A-operand rows of the two accumulators
+  int b_row0;          // first row of the token tile in its tensor map
   int nk;              // 64-wide K steps
-  bool shared;         // shared-expert group (its own weight tensor map)
+  bool shared;         // shared-expert group (its own weight / token tensor maps)
 };
 
 template <int MODE>
-__device__ __forceinline__ Geom tile_geom(const TcArgs& a, const PlanView& pv, int tile) {
+__device__ __forceinline__ Geom tile_geom(const TcArgs& a, const SharedState& S, int tile,
+                                          int R) {
   Geom G;
   if (MODE == kRouter) {
-    // 256 router rows (experts) x up to 256 tokens; K runs over the hi|mid|lo pieces
     const int mt = (a.E + 255) / 256;
     const int m = tile % mt, c = tile / mt;
     G.t.g = 0;
     G.t.m = m;
-    G.t.p0 = c * 256;
-    G.t.nvalid = min(256, a.T - G.t.p0);
+    G.t.p0 = c * kMaxTile;
+    G.t.nvalid = min(kMaxTile, a.T - G.t.p0);
     G.t.N = (G.t.nvalid + 15) & ~15;
     G.a_row0 = m * 256;
     G.a_row1 = m * 256 + 128;
+    G.b_row0 = G.t.p0;
     G.nk = 3 * a.H / 64;
     G.shared = false;
     return G;
   }
-  const int* tp = (MODE == kGateUp) ? pv.tp1 : pv.tp2;
-  G.t = decode_tile(pv, tp, a.E, tile, (MODE == kGateUp) ? kTcChunk : kTcChunkDown);
+  G.t = decode_tile(S.row0, S.tp, a.E, tile);
   G.shared = G.t.g == a.E;
   if (MODE == kGateUp) {
     const int Ig = G.shared ? a.Is : a.I;
     const int base = G.shared ? 0 : G.t.g * 2 * a.I;
     G.a_row0 = base + G.t.m * 128;
     G.a_row1 = base + Ig + G.t.m * 128;
+    G.b_row0 = G.shared ? G.t.p0 - R : G.t.p0;  // x rows for the shared expert
     G.nk = a.H / 64;
   } else {
     const int base = G.shared ? 0 : G.t.g * a.H;
     G.a_row0 = base + G.t.m * 256;
     G.a_row1 = G.a_row0 + 128;
+    G.b_row0 = G.t.p0;
     G.nk = (G.shared ? a.Is : a.I) / 64;
   }
   return G;
@@ -192,36 +209,46 @@ __device__ __forceinline__ Geom tile_geom(const TcArgs& a, const PlanView& pv, i
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_sh,
-                  const __grid_constant__ CUtensorMap tm_b, const TcArgs args) {
+                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b_sh,
+                  const TcArgs args) {
+  using C = Cfg<MODE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  SharedState& S = *reinterpret_cast<SharedState*>(smem + kStages * kStageBytes);
+  SharedState& S = *reinterpret_cast<SharedState*>(smem + C::kStages * C::kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = args.E;
-  PlanView pv{};
   int total, R = 0;
   if (MODE == kRouter) {
     total = args.ntiles;
   } else {
-    pv = plan_view(const_cast<int*>(args.plan), E);
-    total = ((MODE == kGateUp) ? pv.tp1 : pv.tp2)[E + 1];
+    // the plan is read on every tile by every role: keep it in shared memory
+    const PlanView pv = plan_view(const_cast<int*>(args.plan), E);
+    const int* tp = (MODE == kGateUp) ? pv.tp1 : pv.tp2;
+    for (int g = threadIdx.x; g < E + 2; g += blockDim.x) {
+      S.tp[g] = tp[g];
+      S.row0[g] = pv.row0[g];
+    }
+    total = tp[E + 1];
     R = pv.row0[E];
   }
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       ptx::mbar_init(&S.full[s], 1);
       ptx::mbar_init(&S.empty[s], 1);
     }
-    ptx::mbar_init(&S.tmem_full, 1);
-    ptx::mbar_init(&S.tmem_empty, 128);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&S.tmem_full[b], 1);
+      ptx::mbar_init(&S.tmem_empty[b], 128);
+    }
     ptx::mbar_init(&S.drain, 1);
     S.abort = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tm_a);
     ptx::prefetch_tmap(&tm_a_sh);
     ptx::prefetch_tmap(&tm_b);
+    ptx::prefetch_tmap(&tm_b_sh);
   }
   if (warp == 1) {
     ptx::tmem_alloc(&S.tmem_base, kTmemCols);
@@ -234,87 +261,72 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    int it = 0;
-    int armed[kStages];
+    if (lane == 0) {
+      int it = 0;
+      int armed[C::kStages];
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) armed[s] = -1;
-    int aborted = 0;
-    const int plane_rows = (MODE == kDown) ? (int)(args.h_plane / (size_t)args.ldh) : 0;
-    for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
-      const Geom G = tile_geom<MODE>(args, pv, tile);
-      const Tile& tl = G.t;
-      const CUtensorMap* ta = G.shared ? &tm_a_sh : &tm_a;
-      if (MODE == kGateUp) {
-        for (int j = lane; j < tl.N; j += 32) {
-          const int q = j < tl.nvalid ? j : tl.nvalid - 1;  // pad with the last real row
-          S.tok[j] = token_of_row(args, tl.p0 + q, R);
-        }
-        __syncwarp();
-      }
-      if (lane == 0) {
-        const int brows = (MODE == kDown) ? 2 * tl.N : tl.N;
-        const uint32_t bytes = 2 * kATileBytes + (uint32_t)brows * 128u;
+      for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
+      bool aborted = false;
+      const int plane_rows = (MODE == kDown) ? (int)(args.h_plane / (size_t)args.ldh) : 0;
+      for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
+        const Geom G = tile_geom<MODE>(args, S, tile, R);
+        const CUtensorMap* ta = G.shared ? &tm_a_sh : &tm_a;
+        const CUtensorMap* tb = (MODE == kGateUp && G.shared) ? &tm_b_sh : &tm_b;
+        const uint32_t bytes = 2 * kATileBytes + (uint32_t)C::kBTiles * G.t.N * 128u;
         for (int ks = 0; ks < G.nk; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          const int s = it % C::kStages;
+          const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
           if (!wait_phase(&S.empty[s], ph ^ 1u, S, args.status)) {
-            aborted = 1;
+            aborted = true;
             break;
           }
           ptx::mbar_arrive_expect_tx(&S.full[s], bytes);
           armed[s] = (int)ph;
-          uint8_t* st = smem + s * kStageBytes;
+          uint8_t* st = smem + s * C::kStageBytes;
           ptx::tma_load_2d(st, ta, &S.full[s], ks * 64, G.a_row0);
           ptx::tma_load_2d(st + kATileBytes, ta, &S.full[s], ks * 64, G.a_row1);
           uint8_t* b = st + 2 * kATileBytes;
-          if (MODE == kGateUp) {
-            for (int j = 0; j < tl.N; j += 4)
-              ptx::tma_gather4(b + j * 128, &tm_b, &S.full[s], ks * 64, S.tok[j], S.tok[j + 1],
-                               S.tok[j + 2], S.tok[j + 3]);
-          } else if (MODE == kDown) {
-            for (int j = 0; j < tl.N; j += 16) {
-              ptx::tma_load_2d(b + j * 128, &tm_b, &S.full[s], ks * 64, tl.p0 + j);
-              ptx::tma_load_2d(b + (tl.N + j) * 128, &tm_b, &S.full[s], ks * 64,
-                               plane_rows + tl.p0 + j);
-            }
-          } else {
-            const int kx = (ks * 64) % args.H;  // the same x columns for each router piece
-            for (int j = 0; j < tl.N; j += 16)
-              ptx::tma_load_2d(b + j * 128, &tm_b, &S.full[s], kx, tl.p0 + j);
+          const int kx = (MODE == kRouter) ? (ks * 64) % args.H : ks * 64;
+          for (int j = 0; j < G.t.N; j += kBoxRows) {
+            ptx::tma_load_2d(b + j * 128, tb, &S.full[s], kx, G.b_row0 + j);
+            if (MODE == kDown)
+              ptx::tma_load_2d(b + kBTileBytes + j * 128, tb, &S.full[s], kx,
+                               plane_rows + G.b_row0 + j);
           }
         }
       }
-      aborted = __shfl_sync(0xffffffffu, aborted, 0);
-      __syncwarp();
+      if (aborted) {
+        // let this CTA's copies in flight land before the shared memory is released
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed[s] >= 0) drain_phase(&S.full[s], (uint32_t)armed[s]);
+      }
     }
-    if (aborted && lane == 0) {
-      // let this CTA's copies in flight land before the shared memory is released
-      for (int s = 0; s < kStages; ++s)
-        if (armed[s] >= 0) drain_phase(&S.full[s], (uint32_t)armed[s]);
-    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int it = 0, tcount = 0;
       bool aborted = false;
       for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x, ++tcount) {
-        const Geom G = tile_geom<MODE>(args, pv, tile);
-        const int nmma = (MODE == kDown) ? 2 * G.t.N : G.t.N;
-        const uint32_t idesc = ptx::idesc_bf16_f32(128, nmma);
-        if (!wait_phase(&S.tmem_empty, ((uint32_t)tcount & 1u) ^ 1u, S, args.status)) {
+        const Geom G = tile_geom<MODE>(args, S, tile, R);
+        const uint32_t idesc = ptx::idesc_bf16_f32(128, G.t.N);
+        const int buf = tcount & 1;
+        const uint32_t use = (uint32_t)(tcount >> 1) & 1u;  // parity of this buffer's turn
+        if (!wait_phase(&S.tmem_empty[buf], use ^ 1u, S, args.status)) {
           aborted = true;
           break;
         }
         ptx::tc_fence_after();
+        const uint32_t d0 = tmem + buf * kBufCols, d1 = d0 + 128;
         for (int ks = 0; ks < G.nk; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          const int s = it % C::kStages;
+          const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
           if (!wait_phase(&S.full[s], ph, S, args.status)) {
             aborted = true;
             break;
           }
           ptx::tc_fence_after();
-          const uint8_t* st = smem + s * kStageBytes;
+          const uint8_t* st = smem + s * C::kStageBytes;
           const uint64_t a0 = ptx::smem_desc_sw128(st);
           const uint64_t a1 = ptx::smem_desc_sw128(st + kATileBytes);
           const uint64_t bd = ptx::smem_desc_sw128(st + 2 * kATileBytes);
@@ -322,13 +334,18 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
             // +32 bytes along K inside the 128-byte swizzle atom = +2 in the address field
-            ptx::umma_bf16(tmem, a0 + 2 * kk, bd + 2 * kk, idesc, acc);
-            ptx::umma_bf16(tmem + kAcc1Col, a1 + 2 * kk, bd + 2 * kk, idesc, acc);
+            ptx::umma_bf16(d0, a0 + 2 * kk, bd + 2 * kk, idesc, acc);
+            ptx::umma_bf16(d1, a1 + 2 * kk, bd + 2 * kk, idesc, acc);
+            if (MODE == kDown) {  // the lo half of h into the same accumulators
+              const uint64_t bl = bd + (kBTileBytes >> 4);
+              ptx::umma_bf16(d0, a0 + 2 * kk, bl + 2 * kk, idesc, 1u);
+              ptx::umma_bf16(d1, a1 + 2 * kk, bl + 2 * kk, idesc, 1u);
+            }
           }
           ptx::umma_commit(&S.empty[s]);
         }
         if (aborted) break;
-        ptx::umma_commit(&S.tmem_full);
+        ptx::umma_commit(&S.tmem_full[buf]);
       }
       if (aborted) {
         ptx::umma_commit(&S.drain);  // completes once every MMA issued so far is done
@@ -339,98 +356,95 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   } else {
     // ------------------------------------------------------------ epilogue
     const int qd = warp & 3;
-    const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    constexpr int kColChunks = kMaxTile / 32;
     int tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
-      const Geom G = tile_geom<MODE>(args, pv, tile);
+      const Geom G = tile_geom<MODE>(args, S, tile, R);
       const Tile& tl = G.t;
-      const bool ok = wait_phase(&S.tmem_full, (uint32_t)tcount & 1u, S, args.status);
+      const int buf = tcount & 1;
+      const uint32_t use = (uint32_t)(tcount >> 1) & 1u;
+      const uint32_t base = tmem + lane_off + buf * kBufCols;
+      // down: token and weight of columns lane, lane + 32, ... requested before waiting for
+      // the accumulators, so the loads overlap the tile's MMAs
+      int col_tok[kColChunks];
+      float col_w[kColChunks];
+      if (MODE == kDown) {
+#pragma unroll
+        for (int ci = 0; ci < kColChunks; ++ci) {
+          const int c = ci * 32 + lane;
+          col_tok[ci] = 0;
+          col_w[ci] = 0.f;
+          if (c < tl.nvalid) {
+            const int p = tl.p0 + c;
+            col_tok[ci] = token_of_row(args, p, R);
+            if (args.out) col_w[ci] = p < R ? args.sorted_w[p] : args.sgate[col_tok[ci]];
+          }
+        }
+      }
+      const bool ok = wait_phase(&S.tmem_full[buf], use, S, args.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       ptx::tc_fence_after();
-      if (MODE == kGateUp) {
-        const int ch = tl.m * 128 + qd * 32 + lane;
-        for (int c0 = 0; c0 < tl.nvalid; c0 += 32) {
-          uint32_t g[32], u[32];
-          ptx::tmem_ld32(lane_base + c0, g);
-          ptx::tmem_ld32(lane_base + kAcc1Col + c0, u);
-          ptx::tmem_ld_wait();
+#pragma unroll
+      for (int ci = 0; ci < kColChunks; ++ci) {
+        const int c0 = ci * 32;
+        if (c0 >= tl.nvalid) break;
+        uint32_t r0[32], r1[32];
+        ptx::tmem_ld32(base + c0, r0);
+        ptx::tmem_ld32(base + 128 + c0, r1);
+        ptx::tmem_ld_wait();
+        if (MODE == kGateUp) {
+          const int ch = tl.m * 128 + qd * 32 + lane;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (c0 + j < tl.nvalid) {
-              const float gv = __uint_as_float(g[j]);
-              const float hv = gv / (1.f + expf(-gv)) * __uint_as_float(u[j]);
+              const float gv = __uint_as_float(r0[j]);
+              const float hv = gv / (1.f + expf(-gv)) * __uint_as_float(r1[j]);
               const uint16_t hi = f32_to_bf16_rn(hv);
               const size_t at = (size_t)(tl.p0 + c0 + j) * args.ldh + ch;
               args.h[at] = hi;
               args.h[args.h_plane + at] = f32_to_bf16_rn(hv - bf16lo(hi));
             }
           }
-        }
-      } else if (MODE == kRouter) {
-        const int e0 = tl.m * 256 + qd * 32 + lane;  // experts e0 and e0 + 128
-        for (int c0 = 0; c0 < tl.nvalid; c0 += 32) {
-          uint32_t l0[32], l1[32];
-          ptx::tmem_ld32(lane_base + c0, l0);
-          ptx::tmem_ld32(lane_base + kAcc1Col + c0, l1);
-          ptx::tmem_ld_wait();
+        } else if (MODE == kRouter) {
+          const int e0 = tl.m * 256 + qd * 32 + lane;  // experts e0 and e0 + 128
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (c0 + j < tl.nvalid) {
               float* row = args.logits + (size_t)(tl.p0 + c0 + j) * E;
-              if (e0 < E) row[e0] = __uint_as_float(l0[j]);
-              if (e0 + 128 < E) row[e0 + 128] = __uint_as_float(l1[j]);
+              if (e0 < E) row[e0] = __uint_as_float(r0[j]);
+              if (e0 + 128 < E) row[e0 + 128] = __uint_as_float(r1[j]);
             }
           }
-        }
-      } else {
-        const int m = tl.m * 256 + qd * 32 + lane;  // rows m (first accumulator), m + 128
-        const int H = args.H;
-        for (int c0 = 0; c0 < tl.nvalid; c0 += 32) {
-          uint32_t ra[32], rb[32];
-          float y0[32], y1[32];
-          ptx::tmem_ld32(lane_base + c0, ra);
-          ptx::tmem_ld32(lane_base + tl.N + c0, rb);
-          ptx::tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y0[j] = __uint_as_float(ra[j]) + __uint_as_float(rb[j]);
-          ptx::tmem_ld32(lane_base + kAcc1Col + c0, ra);
-          ptx::tmem_ld32(lane_base + kAcc1Col + tl.N + c0, rb);
-          ptx::tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y1[j] = __uint_as_float(ra[j]) + __uint_as_float(rb[j]);
-          // token and weight of column c0 + lane
-          const int colp = tl.p0 + c0 + lane;
-          int tok = 0;
-          float wgt = 0.f;
-          if (c0 + lane < tl.nvalid) {
-            tok = token_of_row(args, colp, R);
-            if (args.out) wgt = colp < R ? args.sorted_w[colp] : args.sgate[tok];
-          }
+        } else {
+          const int m = tl.m * 256 + qd * 32 + lane;  // rows m (first accumulator), m + 128
+          const int H = args.H;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (c0 + j < tl.nvalid) {
-              const int t = __shfl_sync(0xffffffffu, tok, j);
-              const float w = __shfl_sync(0xffffffffu, wgt, j);
+              const float y0 = __uint_as_float(r0[j]), y1 = __uint_as_float(r1[j]);
+              const int t = __shfl_sync(0xffffffffu, col_tok[ci], j);
+              const float w = __shfl_sync(0xffffffffu, col_w[ci], j);
               const int p = tl.p0 + c0 + j;
               if (args.out) {
                 float* o = args.out + (size_t)t * H + m;
-                atomicAdd(o, w * y0[j]);
-                atomicAdd(o + 128, w * y1[j]);
+                atomicAdd(o, w * y0);
+                atomicAdd(o + 128, w * y1);
               } else if (p < R) {
                 float* o = args.y + (size_t)p * H + m;
-                o[0] = y0[j];
-                o[128] = y1[j];
+                o[0] = y0;
+                o[128] = y1;
               } else {
                 float* o = args.y_shared + (size_t)(p - R) * H + m;
-                o[0] = y0[j];
-                o[128] = y1[j];
+                o[0] = y0;
+                o[128] = y1;
               }
             }
           }
         }
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&S.tmem_empty);
+      ptx::mbar_arrive(&S.tmem_empty[buf]);
     }
   }
 
@@ -442,9 +456,30 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   }
 }
 
+// Token rows in dispatch order: xs[p] = x[sorted_token[p]] for the R routed rows, so that
+// a tile's tokens are consecutive rows of one tensor. One warp per row, 16-byte copies.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_token,
+                   const int* __restrict__ plan, int E, int T, int H, uint16_t* __restrict__ xs,
+                   uint32_t* __restrict__ status) {
+  const int R = plan_view(const_cast<int*>(plan), E).row0[E];
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < R; p += nwarps) {
+    int t = sorted_token[p];
+    if ((unsigned)t >= (unsigned)T) {
+      set_flag(status, kFlagBounds);
+      t = 0;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)p * H);
+    for (int c = lane; c < H / 8; c += 32) dst[c] = __ldg(src + c);
+  }
+}
+
 // Router matrix fp32 [E][H] -> bf16 pieces [E][3H] = hi | mid | lo with
 // w = hi + mid + lo exactly (each piece takes the next 8 significant bits), so every
-// product with a bf16 activation is exact and the tensor-core sum is an fp32 dot product.
+// product with a bf16 activation is exact.
 __global__ void router_split_kernel(const float* __restrict__ wr, uint16_t* __restrict__ out,
                                     int E, int H) {
   const size_t n = (size_t)E * H;
@@ -503,15 +538,16 @@ int sm_count() {
 
 template <int MODE>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& a_sh, const CUtensorMap& b,
-                        const TcArgs& args, cudaStream_t st) {
+                        const CUtensorMap& b_sh, const TcArgs& args, int grid, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(tc_grouped_kernel<MODE>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem_bytes<MODE>());
   });
   if (attr_err != cudaSuccess) return attr_err;
-  tc_grouped_kernel<MODE><<<sm_count(), kThreads, kSmemBytes, st>>>(a, a_sh, b, args);
+  tc_grouped_kernel<MODE><<<grid, kThreads, smem_bytes<MODE>(), st>>>(a, a_sh, b, b_sh, args);
   return cudaGetLastError();
 }
 
@@ -553,44 +589,41 @@ cudaError_t launch_tc_router(const moe_shape& s, const Layout& L, char* ws, cons
   }
   CUtensorMap a, b;
   if (!make_map(&a, split, 3ull * s.H, (uint64_t)s.E, 64, 128) ||
-      !make_map(&b, x, s.H, (uint64_t)s.T, 64, 16))
+      !make_map(&b, x, s.H, (uint64_t)s.T, 64, kBoxRows))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.logits = logits;
-  args.ntiles = ((s.E + 255) / 256) * ((s.T + 255) / 256);
+  args.ntiles = ((s.E + 255) / 256) * ((s.T + kMaxTile - 1) / kMaxTile);
   LaunchScope scope(MOE_K_ROUTER_LOGITS, st);
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(tc_grouped_kernel<kRouter>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
-  const int grid = std::min(args.ntiles, sm_count());
-  tc_grouped_kernel<kRouter><<<grid, kThreads, kSmemBytes, st>>>(a, a, b, args);
-  return cudaGetLastError();
+  return launch_mode<kRouter>(a, a, b, b, args, std::min(args.ntiles, sm_count()), st);
 }
 
 bool tc_supported(const moe_shape& s) {
   if (s.I % 128 || s.Is % 128 || s.H % 256) return false;
-  int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-    return false;
-  return major == 10 && encode_fn() != nullptr;
+  return tc_router_supported(s);
 }
 
 cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                               const int32_t* sorted_token, const moe_weights& w, cudaStream_t st) {
-  CUtensorMap a, a_sh, b;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
+  {
+    LaunchScope scope(MOE_K_OTHER, st);
+    gather_rows_kernel<<<sm_count() * 8, 256, 0, st>>>(
+        x, sorted_token, reinterpret_cast<const int*>(ws + L.plan), s.E, s.T, s.H, xs,
+        reinterpret_cast<uint32_t*>(ws + L.status));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap a, a_sh, b, b_sh;
   if (!make_map(&a, w.w_gate_up, s.H, (uint64_t)s.E * 2 * s.I, 64, 128) ||
       !make_map(&a_sh, w.ws_gate_up, s.H, 2ull * s.Is, 64, 128) ||
-      !make_map(&b, x, s.H, (uint64_t)s.T, 64, 1))
+      !make_map(&b, xs, s.H, (uint64_t)s.T * s.k, 64, kBoxRows) ||
+      !make_map(&b_sh, x, s.H, (uint64_t)s.T, 64, kBoxRows))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
   LaunchScope scope(MOE_K_GATE_UP, st);
-  return launch_mode<kGateUp>(a, a_sh, b, args, st);
+  return launch_mode<kGateUp>(a, a_sh, b, b_sh, args, sm_count(), st);
 }
 
 cudaError_t launch_tc_down(const moe_shape& s, const Layout& L, char* ws,
@@ -600,7 +633,7 @@ cudaError_t launch_tc_down(const moe_shape& s, const Layout& L, char* ws,
   CUtensorMap a, a_sh, b;
   if (!make_map(&a, w.w_down, s.I, (uint64_t)s.E * s.H, 64, 128) ||
       !make_map(&a_sh, w.ws_down, s.Is, (uint64_t)s.H, 64, 128) ||
-      !make_map(&b, ws + L.h, L.ldh, 2 * (L.h_plane / L.ldh), 64, 16))
+      !make_map(&b, ws + L.h, L.ldh, 2 * (L.h_plane / L.ldh), 64, kBoxRows))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
@@ -610,7 +643,7 @@ cudaError_t launch_tc_down(const moe_shape& s, const Layout& L, char* ws,
   args.y_shared = y_shared;
   args.out = out;
   LaunchScope scope(MOE_K_DOWN, st);
-  return launch_mode<kDown>(a, a_sh, b, args, st);
+  return launch_mode<kDown>(a, a_sh, b, b, args, sm_count(), st);
 }
 
 }  // namespace moe
