@@ -38,6 +38,7 @@ Layout layout(const moe_shape& s) {
   L.sorted_w = take(R * sizeof(float));
   L.assign_row = take(R * sizeof(int32_t));
   L.plan = take(plan_ints(s.E) * sizeof(int32_t));
+  L.sched = take(4 * sizeof(int32_t));
   L.xs = take(R * H * sizeof(uint16_t));
   L.h_plane = (R + T) * (size_t)L.ldh;
   L.h = take(2 * L.h_plane * sizeof(uint16_t));

@@ -35,6 +35,8 @@ struct Layout {
   size_t sorted_w;      // fp32 [T*k]: routing weight of each packed row
   size_t assign_row;    // int32 [T*k]
   size_t plan;          // int32 plan arrays (see PlanView)
+  size_t sched;         // int32 [4] tile counters of the tensor-core kernels (gate|up, down,
+                        // router), zeroed by the kernel that runs before each of them
   size_t xs;            // bf16 [T*k][H]: token rows in dispatch order (tensor-core gate|up)
   size_t h;             // bf16 [2][T*k + T][ldh]: SwiGLU intermediate as a hi|lo pair of planes
                         // (h = hi + lo), routed rows then shared rows

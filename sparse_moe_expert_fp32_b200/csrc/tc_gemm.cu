@@ -61,14 +61,19 @@ struct Cfg {
   static constexpr int kStages = (MODE == kDown) ? 3 : 4;
 };
 
+constexpr int kQueue = 4;  // tile ids handed from the producer to the MMA and epilogue roles
+
 struct SharedState {
   uint64_t full[4];
   uint64_t empty[4];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
+  uint64_t q_full[kQueue];
+  uint64_t q_empty[kQueue];
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort;
+  int q[kQueue];
   int tp[kMaxE + 2];    // tile prefix of the grouped GEMM (copied from the plan)
   int row0[kMaxE + 2];  // first packed row of each group (copied from the plan)
 };
@@ -92,6 +97,8 @@ struct TcArgs {
   uint32_t* status;
   float* logits;  // router: [T][E]
   int ntiles;     // router: tile count (no plan)
+  int* counter;   // next tile to hand out (zeroed before the launch)
+  int* counter_next;  // gate|up: the down kernel's counter, zeroed here for the next launch
 };
 
 struct Tile {
@@ -233,6 +240,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     R = pv.row0[E];
   }
 
+  if (MODE == kGateUp && blockIdx.x == 0 && threadIdx.x == 0) *args.counter_next = 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       ptx::mbar_init(&S.full[s], 1);
@@ -241,6 +249,10 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&S.tmem_full[b], 1);
       ptx::mbar_init(&S.tmem_empty[b], 128);
+    }
+    for (int i = 0; i < kQueue; ++i) {
+      ptx::mbar_init(&S.q_full[i], 1);
+      ptx::mbar_init(&S.q_empty[i], 5);  // the MMA lane and one lane of each epilogue warp
     }
     ptx::mbar_init(&S.drain, 1);
     S.abort = 0;
@@ -268,7 +280,19 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
       bool aborted = false;
       const int plane_rows = (MODE == kDown) ? (int)(args.h_plane / (size_t)args.ldh) : 0;
-      for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
+      // tiles are handed out in order by one counter: the token chunks of one weight tile
+      // start together on neighbouring SMs, so the second read of the weights hits L2
+      for (int qi = 0; !aborted; ++qi) {
+        const int slot = qi % kQueue;
+        if (!wait_phase(&S.q_empty[slot], ((uint32_t)(qi / kQueue) & 1u) ^ 1u, S, args.status)) {
+          aborted = true;
+          break;
+        }
+        int tile = atomicAdd(args.counter, 1);
+        if (tile >= total) tile = -1;
+        S.q[slot] = tile;
+        ptx::mbar_arrive(&S.q_full[slot]);
+        if (tile < 0) break;
         const Geom G = tile_geom<MODE>(args, S, tile, R);
         const CUtensorMap* ta = G.shared ? &tm_a_sh : &tm_a;
         const CUtensorMap* tb = (MODE == kGateUp && G.shared) ? &tm_b_sh : &tm_b;
@@ -307,7 +331,15 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     if (lane == 0) {
       int it = 0, tcount = 0;
       bool aborted = false;
-      for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x, ++tcount) {
+      for (int qi = 0; !aborted; ++qi, ++tcount) {
+        const int slot = qi % kQueue;
+        if (!wait_phase(&S.q_full[slot], (uint32_t)(qi / kQueue) & 1u, S, args.status)) {
+          aborted = true;
+          break;
+        }
+        const int tile = S.q[slot];
+        ptx::mbar_arrive(&S.q_empty[slot]);
+        if (tile < 0) break;
         const Geom G = tile_geom<MODE>(args, S, tile, R);
         const uint32_t idesc = ptx::idesc_bf16_f32(128, G.t.N);
         const int buf = tcount & 1;
@@ -359,7 +391,14 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     constexpr int kColChunks = kMaxTile / 32;
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+    for (int qi = 0;; ++qi, ++tcount) {
+      const int slot = qi % kQueue;
+      const bool got = wait_phase(&S.q_full[slot], (uint32_t)(qi / kQueue) & 1u, S, args.status);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const int tile = S.q[slot];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&S.q_empty[slot]);
+      if (tile < 0) break;
       const Geom G = tile_geom<MODE>(args, S, tile, R);
       const Tile& tl = G.t;
       const int buf = tcount & 1;
@@ -399,7 +438,9 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           for (int j = 0; j < 32; ++j) {
             if (c0 + j < tl.nvalid) {
               const float gv = __uint_as_float(r0[j]);
-              const float hv = gv / (1.f + expf(-gv)) * __uint_as_float(r1[j]);
+              // SiLU(g) = g / (1 + e^-g) with the fast exponential and division (a few ulp;
+              // h is carried with about 16 significant bits)
+              const float hv = __fdividef(gv, 1.f + __expf(-gv)) * __uint_as_float(r1[j]);
               const uint16_t hi = f32_to_bf16_rn(hv);
               const size_t at = (size_t)(tl.p0 + c0 + j) * args.ldh + ch;
               args.h[at] = hi;
@@ -461,7 +502,8 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ sorted_token,
                    const int* __restrict__ plan, int E, int T, int H, uint16_t* __restrict__ xs,
-                   uint32_t* __restrict__ status) {
+                   uint32_t* __restrict__ status, int* __restrict__ counter) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *counter = 0;  // tile counter of the gate|up GEMM
   const int R = plan_view(const_cast<int*>(plan), E).row0[E];
   const int lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -481,7 +523,8 @@ gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ s
 // w = hi + mid + lo exactly (each piece takes the next 8 significant bits), so every
 // product with a bf16 activation is exact.
 __global__ void router_split_kernel(const float* __restrict__ wr, uint16_t* __restrict__ out,
-                                    int E, int H) {
+                                    int E, int H, int* __restrict__ counter) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *counter = 0;  // tile counter of the router GEMM
   const size_t n = (size_t)E * H;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -583,7 +626,8 @@ cudaError_t launch_tc_router(const moe_shape& s, const Layout& L, char* ws, cons
     LaunchScope scope(MOE_K_OTHER, st);
     const size_t n = (size_t)s.E * s.H;
     const int blocks = (int)std::min<size_t>((n + 255) / 256, (size_t)sm_count() * 8);
-    router_split_kernel<<<blocks, 256, 0, st>>>(wr, split, s.E, s.H);
+    router_split_kernel<<<blocks, 256, 0, st>>>(wr, split, s.E, s.H,
+                                                reinterpret_cast<int*>(ws + L.sched) + 2);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -593,6 +637,7 @@ cudaError_t launch_tc_router(const moe_shape& s, const Layout& L, char* ws, cons
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.logits = logits;
+  args.counter = reinterpret_cast<int*>(ws + L.sched) + 2;
   args.ntiles = ((s.E + 255) / 256) * ((s.T + kMaxTile - 1) / kMaxTile);
   LaunchScope scope(MOE_K_ROUTER_LOGITS, st);
   return launch_mode<kRouter>(a, a, b, b, args, std::min(args.ntiles, sm_count()), st);
@@ -610,7 +655,7 @@ cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, con
     LaunchScope scope(MOE_K_OTHER, st);
     gather_rows_kernel<<<sm_count() * 8, 256, 0, st>>>(
         x, sorted_token, reinterpret_cast<const int*>(ws + L.plan), s.E, s.T, s.H, xs,
-        reinterpret_cast<uint32_t*>(ws + L.status));
+        reinterpret_cast<uint32_t*>(ws + L.status), reinterpret_cast<int*>(ws + L.sched) + 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -622,6 +667,8 @@ cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, con
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
+  args.counter = reinterpret_cast<int*>(ws + L.sched) + 0;
+  args.counter_next = reinterpret_cast<int*>(ws + L.sched) + 1;
   LaunchScope scope(MOE_K_GATE_UP, st);
   return launch_mode<kGateUp>(a, a_sh, b, b_sh, args, sm_count(), st);
 }
@@ -642,6 +689,7 @@ cudaError_t launch_tc_down(const moe_shape& s, const Layout& L, char* ws,
   args.y = y;
   args.y_shared = y_shared;
   args.out = out;
+  args.counter = reinterpret_cast<int*>(ws + L.sched) + 1;
   LaunchScope scope(MOE_K_DOWN, st);
   return launch_mode<kDown>(a, a_sh, b, b, args, sm_count(), st);
 }

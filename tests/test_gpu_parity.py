@@ -124,7 +124,7 @@ def test_router_topk_parity(name):
     g = gap.cpu().numpy()
     assert (g >= 0).all()
     # near the decision the kernel recomputes logits exactly: tight there, loose elsewhere
-    near = [t for t in same if rgap[t] < 2e-3]
+    near = [t for t in same if rgap[t] < 1e-3]
     assert np.allclose(g[near], rgap[near], atol=5e-5)
     assert np.allclose(g[same], rgap[same], atol=1e-3)
 
