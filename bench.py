@@ -263,16 +263,17 @@ def run_reference(args, cfg, world, rank):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_block(cfg, None),
+            "config": config_block(cfg, None, "fp64 oracle on the host cores"),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def config_block(cfg, variant):
+def config_block(cfg, variant, timed_as="CUDA graph replay of one layer forward per step"):
     return {"workload": cfg.name, "description": cfg.description, "T": cfg.T, "H": cfg.H, "E": cfg.E,
             "k": cfg.k, "I": cfg.I, "Is": cfg.Is, "zipf_s": cfg.zipf_s, "zero_rows_pct": cfg.zero_rows_pct,
             "variant": variant, "accumulate": "fp32", "output": "fp32",
+            "timed_as": timed_as,
             "l2": "inputs larger than L2 (expert weight bank exceeds the 126 MB L2)"
             if cfg.E * 3 * cfg.H * cfg.I * 2 > 126e6 else "L2-resident (tiny layer)",
             "parallelism": "replicas: one token batch per GPU, no collective"}
@@ -326,25 +327,48 @@ def run_ours(args, cfg, world, rank, local):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    # ---- device-resident timed region
+    # ---- device-resident timed region: one layer forward per step, replayed from a CUDA
+    # graph (as a served layer would run; --no-graph launches every kernel from the host)
     windows = []
+    graph = None
+    moe.moe_profile_enable(True)  # fill the library's event pool before any capture
+    moe.moe_layer_forward(s, dev["x"], w, out, ws)
+    torch.cuda.synchronize()
+    moe.moe_profile_collect()
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        n_cap = moe.moe_launch_count()
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            moe.moe_layer_forward(s, dev["x"], w, out, ws)
+        per_step = moe.moe_launch_count() - n_cap
+        stream = torch.cuda.current_stream()
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    moe.moe_profile_enable(True)
     n0 = moe.moe_launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     w0 = time.time()
     e0.record(stream)
     for _ in range(args.steps):
-        moe.moe_layer_forward(s, dev["x"], w, out, ws)
+        if graph is not None:
+            graph.replay()
+        else:
+            moe.moe_layer_forward(s, dev["x"], w, out, ws)
     e1.record(stream)
     torch.cuda.synchronize()
     windows.append((w0, time.time()))
-    launches = moe.moe_launch_count() - n0
+    launches = per_step * args.steps if graph is not None else moe.moe_launch_count() - n0
     moe.moe_profile_enable(False)
+    # per-kernel device times: every launch of the timed region, or, with the graph, the
+    # event nodes of its last replay (every replay runs the same kernels on the same data)
     prof = moe.moe_profile_collect()
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1))
+    st, flags = moe.moe_device_status(ws)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after the timed region {st} ({flags})")
 
     # ---- end to end through the host-buffer entry point
     x_host = dev["x"].cpu().pin_memory()
@@ -397,7 +421,11 @@ def run_ours(args, cfg, world, rank, local):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "us_per_layer": 1e3 * ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random router)",
-            "config": config_block(cfg, args.variant), "roofline": roofline,
+            "config": config_block(cfg, args.variant,
+                                   "host launches of one layer forward per step" if args.no_graph
+                                   else "CUDA graph replay of one layer forward per step"),
+            "roofline": roofline,
+            "graph": not args.no_graph,
             "e2e": {"value": cfg.T * args.steps * world / (ms_e2e / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 4},
             "gpu_launches": launches, "kernels": kernels,
@@ -418,6 +446,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto", choices=["auto", "stream", "tc"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every kernel from the host")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = synth.CONFIGS[args.workload]
