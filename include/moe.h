@@ -213,7 +213,8 @@ moe_status moe_debug_wait_flag(const int32_t* flag, uint64_t timeout_ns, void* w
                                size_t ws_bytes, void* stream);
 
 /* Measurement: while enabled, every kernel launch records a CUDA event pair on its
- * stream. moe_profile_collect synchronises those events and returns, per moe_kernel
+ * stream (launches into a stream that is being captured into a CUDA graph are not
+ * recorded). moe_profile_collect synchronises those events and returns, per moe_kernel
  * id, the summed device time in ms (HOST float[MOE_K_COUNT]) and the launch counts
  * (HOST int32[MOE_K_COUNT]), then forgets them. At most 65536 launches are recorded. */
 moe_status moe_profile_enable(int32_t on);

@@ -78,6 +78,8 @@ cudaEvent_t pool_event() {
 LaunchScope::LaunchScope(moe_kernel id, cudaStream_t s, int nkernels) : slot(-1), stream(s) {
   g_launches.fetch_add((uint64_t)nkernels, std::memory_order_relaxed);
   if (!g_prof_on) return;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (!g_prof_on || g_recs.size() >= kMaxProfRecs) return;
   cudaEvent_t a = pool_event(), b = pool_event();
