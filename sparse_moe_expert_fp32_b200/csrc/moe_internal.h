@@ -13,7 +13,7 @@ namespace moe {
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 32;
 constexpr int kPermBlock = 256;  // tokens per dispatch block (one bit per token in a mask)
-constexpr int kTcChunk = 128;    // max tokens (MMA N) per tensor-core tile
+constexpr int kTcChunk = 256;    // max tokens (MMA N) per tensor-core tile
 constexpr uint32_t kFlagBounds = 1u;
 constexpr uint32_t kFlagTimeout = 2u;
 
@@ -72,7 +72,7 @@ __host__ __device__ inline PlanView plan_view(void* base, int E) {
 }
 
 // Tensor-core tiling of a group with n rows into ceil(n / max) token chunks of nearly equal
-// size (multiples of 16 rows), max 128 rows for both grouped GEMMs.
+// size (multiples of 16 rows), max 256 rows for both grouped GEMMs.
 constexpr int kTcChunkDown = kTcChunk;
 __host__ __device__ inline int tc_nchunks(int n, int max_rows) {
   return (n + max_rows - 1) / max_rows;

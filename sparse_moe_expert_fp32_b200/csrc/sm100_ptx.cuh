@@ -140,15 +140,23 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Shared-memory matrix descriptor: K-major operand staged by TMA with 128-byte swizzle,
-// rows of 128 bytes (64 bf16), 8-row groups 1024 bytes apart (stride byte offset).
-// Fields: start address >> 4 [0,14), leading byte offset >> 4 [16,30) (0: unused for
-// swizzled K-major), stride byte offset >> 4 [32,46), version 1 [46,48),
-// base offset 0 (1024-byte aligned atoms), layout type 2 = 128-byte swizzle [61,64).
-__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
+// Shared-memory matrix descriptor of a K-major operand staged by TMA with a 128-byte
+// (rows of 64 bf16) or 64-byte (rows of 32 bf16) swizzle: 8-row groups are 8 rows apart
+// (stride byte offset 1024 or 512). Fields: start address >> 4 [0,14), leading byte
+// offset >> 4 [16,30) (0: unused for swizzled K-major), stride byte offset >> 4 [32,46),
+// version 1 [46,48), base offset 0 (atoms aligned to their size), layout type [61,64):
+// 2 = 128-byte swizzle, 4 = 64-byte swizzle.
+template <int kRowBytes>
+__device__ __forceinline__ uint64_t smem_desc_kmajor(const void* p) {
+  static_assert(kRowBytes == 128 || kRowBytes == 64, "128- or 64-byte swizzle");
   const uint64_t addr = smem_u32(p);
-  return ((addr >> 4) & 0x3FFFull) | ((1024ull >> 4) << 32) | (1ull << 46) |
-         (2ull << 61);
+  const uint64_t layout = kRowBytes == 128 ? 2ull : 4ull;
+  return ((addr >> 4) & 0x3FFFull) | ((uint64_t)(8 * kRowBytes) >> 4 << 32) | (1ull << 46) |
+         (layout << 61);
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
+  return smem_desc_kmajor<128>(p);
 }
 
 // Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major.

@@ -5,27 +5,31 @@
 //
 // Orientation ("swap AB"): weight rows are the MMA's M side (two 128-row accumulators per
 // tile = 256 weight rows sharing one token tile), the tokens of one expert are the N side
-// (multiples of 16, at most 128 per tile), K is the hidden (gate|up, router) or
-// intermediate (down) dimension. Every weight byte comes from HBM once per token chunk;
-// the chunks of one weight tile are neighbouring tiles, so a second chunk reads it from L2.
+// (multiples of 16, up to 256 per tile, so a prefill expert is one tile and its weights
+// pass through shared memory once), K is the hidden (gate|up, router) or intermediate
+// (down) dimension.
 //
 //   gate|up: gate rows [c, c+128) and up rows [I+c, I+c+128) of one expert against its
 //     token rows, copied beforehand in dispatch order (gather_rows_kernel) so that a token
 //     tile is a few plain 2-D TMA boxes. Epilogue: h = SiLU(gate) * up stored as the bf16
 //     pair hi = bf16(h), lo = bf16(h - hi).
 //   down: 256 rows of one expert's W_down against its packed rows; per K step two MMAs add
-//     W h_hi and W h_lo into the same accumulators. Epilogue: y rows (staged path) or
+//     W h_hi and W h_lo into the same accumulators (32-wide K stages, 64-byte swizzle, so
+//     that a 256-token tile still leaves four stages). Epilogue: y rows (staged path) or
 //     routing-weight-scaled fp32 atomic adds into out[token] ("Weighted combine + gated
 //     shared expert").
 //   router: 256 experts x 128 tokens of logits = x . (hi + mid + lo)^T, K = 3H over the
 //     exact bf16 split of the fp32 router matrix.
 //
-// Roles in a 192-thread CTA (one CTA per SM, persistent over the tile list):
+// Roles in a 320-thread CTA (one CTA per SM, persistent; tiles handed out in order by an
+// atomic counter through a shared-memory queue):
 //   warp 0      TMA producer (lane 0 issues) over a ring of kStages stages;
-//   warp 1      TMEM owner (all 512 columns = two accumulator buffers of 2 x 128 columns)
-//               and MMA issuer (lane 0);
-//   warps 2..5  epilogue, warp w reads TMEM lanes 32*(w%4) .. +31; while it drains one
-//               buffer the MMAs of the next tile fill the other.
+//   warp 1      TMEM owner (all 512 columns, two slots of 256) and MMA issuer (lane 0);
+//               a tile of at most 128 tokens takes one slot (its two accumulators are
+//               128 columns each) and the next tile's MMAs fill the other slot while the
+//               epilogue drains it; a larger tile takes both slots;
+//   warps 2..9  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31, the first four warps
+//               even 32-column chunks, the last four odd ones.
 // Every mbarrier wait is bounded (2 s); on expiry the kernel records the timeout flag,
 // lets every role leave its loop, drains its own copies and MMAs and frees TMEM.
 #include <cuda.h>
@@ -41,27 +45,30 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr uint32_t kATileBytes = 128 * 128;   // 128 rows x 64 bf16
-constexpr uint32_t kBTileBytes = 128 * 128;   // up to 128 token rows x 64 bf16
-constexpr int kBoxRows = 16;                  // rows per TMA box of a token tile
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kBoxRows = 16;  // rows per TMA box of a token tile
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kBufCols = 256;  // one accumulator buffer: two 128-column accumulators
-constexpr int kMaxTile = 128;       // tokens per tile (MMA N)
+constexpr uint32_t kSlotCols = 256;
+constexpr int kQueue = 4;  // tile ids handed from the producer to the MMA and epilogue roles
 
 enum Mode { kGateUp = 0, kDown = 1, kRouter = 2 };
 
-// Stage = two A tiles + one (gate|up, router) or two (down: hi, lo) token tiles.
+// Per-mode pipeline geometry.
 template <int MODE>
 struct Cfg {
-  static constexpr int kBTiles = (MODE == kDown) ? 2 : 1;
+  static constexpr int kBK = (MODE == kDown) ? 32 : 64;        // K per stage
+  static constexpr int kRowBytes = kBK * 2;                      // 64 or 128 (= swizzle)
+  static constexpr int kMaxTile = (MODE == kRouter) ? 128 : 256;  // tokens per tile
+  static constexpr uint32_t kATileBytes = 128u * kRowBytes;
+  static constexpr uint32_t kBTileBytes = (uint32_t)kMaxTile * kRowBytes;
+  static constexpr int kBTiles = (MODE == kDown) ? 2 : 1;  // down: hi and lo rows of h
   static constexpr uint32_t kStageBytes = 2 * kATileBytes + kBTiles * kBTileBytes;
-  static constexpr int kStages = (MODE == kDown) ? 3 : 4;
+  static constexpr int kStages = (MODE == kDown) ? 4 : 3;
+  static constexpr int kKK = kBK / 16;  // MMAs (K = 16) per stage and accumulator
 };
-
-constexpr int kQueue = 4;  // tile ids handed from the producer to the MMA and epilogue roles
 
 struct SharedState {
   uint64_t full[4];
@@ -95,10 +102,10 @@ struct TcArgs {
   float* y_shared;
   float* out;
   uint32_t* status;
-  float* logits;  // router: [T][E]
-  int ntiles;     // router: tile count (no plan)
-  int* counter;   // next tile to hand out (zeroed before the launch)
-  int* counter_next;  // gate|up: the down kernel's counter, zeroed here for the next launch
+  float* logits;      // router: [T][E]
+  int ntiles;         // router: tile count (no plan)
+  int* counter;       // next tile to hand out (zeroed before the launch)
+  int* counter_next;  // gate|up: the down kernel's counter, zeroed here for its launch
 };
 
 struct Tile {
@@ -106,8 +113,10 @@ struct Tile {
 };
 
 // Tile -> (group, M tile, packed rows). Groups own consecutive tile ranges
-// [tp[g], tp[g+1]); inside a group the token chunks of one M tile are adjacent.
-__device__ __forceinline__ Tile decode_tile(const int* row0, const int* tp, int E, int tile) {
+// [tp[g], tp[g+1]); a group of more than max_tile rows is split into near-equal chunks
+// whose tiles are adjacent.
+__device__ __forceinline__ Tile decode_tile(const int* row0, const int* tp, int E, int tile,
+                                            int max_tile) {
   int lo = 0, hi = E + 1;  // tp[lo] <= tile < tp[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -117,7 +126,7 @@ __device__ __forceinline__ Tile decode_tile(const int* row0, const int* tp, int 
   Tile t;
   t.g = lo;
   const int n = row0[lo + 1] - row0[lo];
-  const int nch = (n + kMaxTile - 1) / kMaxTile;
+  const int nch = (n + max_tile - 1) / max_tile;
   const int cs = (((n + nch - 1) / nch) + 15) & ~15;
   const int local = tile - tp[lo];
   t.m = local / nch;
@@ -171,30 +180,31 @@ struct Geom {
   Tile t;
   int a_row0, a_row1;  // A-operand rows of the two accumulators
   int b_row0;          // first row of the token tile in its tensor map
-  int nk;              // 64-wide K steps
+  int nk;              // K stages
   bool shared;         // shared-expert group (its own weight / token tensor maps)
 };
 
 template <int MODE>
 __device__ __forceinline__ Geom tile_geom(const TcArgs& a, const SharedState& S, int tile,
                                           int R) {
+  using C = Cfg<MODE>;
   Geom G;
   if (MODE == kRouter) {
     const int mt = (a.E + 255) / 256;
     const int m = tile % mt, c = tile / mt;
     G.t.g = 0;
     G.t.m = m;
-    G.t.p0 = c * kMaxTile;
-    G.t.nvalid = min(kMaxTile, a.T - G.t.p0);
+    G.t.p0 = c * C::kMaxTile;
+    G.t.nvalid = min(C::kMaxTile, a.T - G.t.p0);
     G.t.N = (G.t.nvalid + 15) & ~15;
     G.a_row0 = m * 256;
     G.a_row1 = m * 256 + 128;
     G.b_row0 = G.t.p0;
-    G.nk = 3 * a.H / 64;
+    G.nk = 3 * a.H / C::kBK;
     G.shared = false;
     return G;
   }
-  G.t = decode_tile(S.row0, S.tp, a.E, tile);
+  G.t = decode_tile(S.row0, S.tp, a.E, tile, C::kMaxTile);
   G.shared = G.t.g == a.E;
   if (MODE == kGateUp) {
     const int Ig = G.shared ? a.Is : a.I;
@@ -202,16 +212,31 @@ __device__ __forceinline__ Geom tile_geom(const TcArgs& a, const SharedState& S,
     G.a_row0 = base + G.t.m * 128;
     G.a_row1 = base + Ig + G.t.m * 128;
     G.b_row0 = G.shared ? G.t.p0 - R : G.t.p0;  // x rows for the shared expert
-    G.nk = a.H / 64;
+    G.nk = a.H / C::kBK;
   } else {
     const int base = G.shared ? 0 : G.t.g * a.H;
     G.a_row0 = base + G.t.m * 256;
     G.a_row1 = G.a_row0 + 128;
     G.b_row0 = G.t.p0;
-    G.nk = (G.shared ? a.Is : a.I) / 64;
+    G.nk = (G.shared ? a.Is : a.I) / C::kBK;
   }
   return G;
 }
+
+// TMEM slot bookkeeping shared by the MMA issuer and the epilogue (both walk the same tile
+// sequence): a tile of at most 128 tokens takes the next slot, a larger one both slots.
+struct Slots {
+  int next = 0;
+  uint32_t uses[2] = {0u, 0u};
+  __device__ __forceinline__ void take(int N, int& first, int& count) const {
+    count = N > 128 ? 2 : 1;
+    first = count == 2 ? 0 : next;
+  }
+  __device__ __forceinline__ void done(int first, int count) {
+    for (int i = 0; i < count; ++i) uses[(first + i) & 1]++;
+    next = count == 2 ? 0 : (first ^ 1);
+  }
+};
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -248,11 +273,11 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&S.tmem_full[b], 1);
-      ptx::mbar_init(&S.tmem_empty[b], 128);
+      ptx::mbar_init(&S.tmem_empty[b], 32 * kEpiWarps);
     }
     for (int i = 0; i < kQueue; ++i) {
       ptx::mbar_init(&S.q_full[i], 1);
-      ptx::mbar_init(&S.q_empty[i], 5);  // the MMA lane and one lane of each epilogue warp
+      ptx::mbar_init(&S.q_empty[i], 1 + kEpiWarps);  // the MMA lane, one lane per epilogue warp
     }
     ptx::mbar_init(&S.drain, 1);
     S.abort = 0;
@@ -280,8 +305,8 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
       bool aborted = false;
       const int plane_rows = (MODE == kDown) ? (int)(args.h_plane / (size_t)args.ldh) : 0;
-      // tiles are handed out in order by one counter: the token chunks of one weight tile
-      // start together on neighbouring SMs, so the second read of the weights hits L2
+      // tiles are handed out in order by one counter: neighbouring tiles (the chunks of one
+      // weight tile, the M tiles of one expert) run at the same time on neighbouring SMs
       for (int qi = 0; !aborted; ++qi) {
         const int slot = qi % kQueue;
         if (!wait_phase(&S.q_empty[slot], ((uint32_t)(qi / kQueue) & 1u) ^ 1u, S, args.status)) {
@@ -296,7 +321,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         const Geom G = tile_geom<MODE>(args, S, tile, R);
         const CUtensorMap* ta = G.shared ? &tm_a_sh : &tm_a;
         const CUtensorMap* tb = (MODE == kGateUp && G.shared) ? &tm_b_sh : &tm_b;
-        const uint32_t bytes = 2 * kATileBytes + (uint32_t)C::kBTiles * G.t.N * 128u;
+        const uint32_t bytes = 2 * C::kATileBytes + (uint32_t)C::kBTiles * G.t.N * C::kRowBytes;
         for (int ks = 0; ks < G.nk; ++ks, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
@@ -307,14 +332,15 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           ptx::mbar_arrive_expect_tx(&S.full[s], bytes);
           armed[s] = (int)ph;
           uint8_t* st = smem + s * C::kStageBytes;
-          ptx::tma_load_2d(st, ta, &S.full[s], ks * 64, G.a_row0);
-          ptx::tma_load_2d(st + kATileBytes, ta, &S.full[s], ks * 64, G.a_row1);
-          uint8_t* b = st + 2 * kATileBytes;
-          const int kx = (MODE == kRouter) ? (ks * 64) % args.H : ks * 64;
+          const int ka = ks * C::kBK;
+          ptx::tma_load_2d(st, ta, &S.full[s], ka, G.a_row0);
+          ptx::tma_load_2d(st + C::kATileBytes, ta, &S.full[s], ka, G.a_row1);
+          uint8_t* b = st + 2 * C::kATileBytes;
+          const int kx = (MODE == kRouter) ? ka % args.H : ka;
           for (int j = 0; j < G.t.N; j += kBoxRows) {
-            ptx::tma_load_2d(b + j * 128, tb, &S.full[s], kx, G.b_row0 + j);
+            ptx::tma_load_2d(b + j * C::kRowBytes, tb, &S.full[s], kx, G.b_row0 + j);
             if (MODE == kDown)
-              ptx::tma_load_2d(b + kBTileBytes + j * 128, tb, &S.full[s], kx,
+              ptx::tma_load_2d(b + C::kBTileBytes + j * C::kRowBytes, tb, &S.full[s], kx,
                                plane_rows + G.b_row0 + j);
           }
         }
@@ -329,9 +355,10 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int it = 0, tcount = 0;
+      int it = 0;
+      Slots sl;
       bool aborted = false;
-      for (int qi = 0; !aborted; ++qi, ++tcount) {
+      for (int qi = 0; !aborted; ++qi) {
         const int slot = qi % kQueue;
         if (!wait_phase(&S.q_full[slot], (uint32_t)(qi / kQueue) & 1u, S, args.status)) {
           aborted = true;
@@ -342,14 +369,17 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (tile < 0) break;
         const Geom G = tile_geom<MODE>(args, S, tile, R);
         const uint32_t idesc = ptx::idesc_bf16_f32(128, G.t.N);
-        const int buf = tcount & 1;
-        const uint32_t use = (uint32_t)(tcount >> 1) & 1u;  // parity of this buffer's turn
-        if (!wait_phase(&S.tmem_empty[buf], use ^ 1u, S, args.status)) {
-          aborted = true;
-          break;
+        int first, count;
+        sl.take(G.t.N, first, count);
+        for (int i = 0; i < count && !aborted; ++i) {
+          const int sidx = (first + i) & 1;
+          if (!wait_phase(&S.tmem_empty[sidx], (sl.uses[sidx] & 1u) ^ 1u, S, args.status))
+            aborted = true;
         }
+        if (aborted) break;
         ptx::tc_fence_after();
-        const uint32_t d0 = tmem + buf * kBufCols, d1 = d0 + 128;
+        const uint32_t d0 = tmem + first * kSlotCols;
+        const uint32_t d1 = d0 + (count == 2 ? kSlotCols : 128u);
         for (int ks = 0; ks < G.nk; ++ks, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
@@ -359,17 +389,17 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           }
           ptx::tc_fence_after();
           const uint8_t* st = smem + s * C::kStageBytes;
-          const uint64_t a0 = ptx::smem_desc_sw128(st);
-          const uint64_t a1 = ptx::smem_desc_sw128(st + kATileBytes);
-          const uint64_t bd = ptx::smem_desc_sw128(st + 2 * kATileBytes);
+          const uint64_t a0 = ptx::smem_desc_kmajor<C::kRowBytes>(st);
+          const uint64_t a1 = ptx::smem_desc_kmajor<C::kRowBytes>(st + C::kATileBytes);
+          const uint64_t bd = ptx::smem_desc_kmajor<C::kRowBytes>(st + 2 * C::kATileBytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < C::kKK; ++kk) {
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-            // +32 bytes along K inside the 128-byte swizzle atom = +2 in the address field
+            // +32 bytes along K inside the swizzle atom = +2 in the address field
             ptx::umma_bf16(d0, a0 + 2 * kk, bd + 2 * kk, idesc, acc);
             ptx::umma_bf16(d1, a1 + 2 * kk, bd + 2 * kk, idesc, acc);
             if (MODE == kDown) {  // the lo half of h into the same accumulators
-              const uint64_t bl = bd + (kBTileBytes >> 4);
+              const uint64_t bl = bd + (C::kBTileBytes >> 4);
               ptx::umma_bf16(d0, a0 + 2 * kk, bl + 2 * kk, idesc, 1u);
               ptx::umma_bf16(d1, a1 + 2 * kk, bl + 2 * kk, idesc, 1u);
             }
@@ -377,7 +407,8 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           ptx::umma_commit(&S.empty[s]);
         }
         if (aborted) break;
-        ptx::umma_commit(&S.tmem_full[buf]);
+        for (int i = 0; i < count; ++i) ptx::umma_commit(&S.tmem_full[(first + i) & 1]);
+        sl.done(first, count);
       }
       if (aborted) {
         ptx::umma_commit(&S.drain);  // completes once every MMA issued so far is done
@@ -388,10 +419,11 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   } else {
     // ------------------------------------------------------------ epilogue
     const int qd = warp & 3;
+    const int half = (warp - 2) / 4;  // which 32-column chunks this warp drains
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    constexpr int kColChunks = kMaxTile / 32;
-    int tcount = 0;
-    for (int qi = 0;; ++qi, ++tcount) {
+    constexpr int kChunks = Cfg<MODE>::kMaxTile / 64;  // chunks per warp
+    Slots sl;
+    for (int qi = 0;; ++qi) {
       const int slot = qi % kQueue;
       const bool got = wait_phase(&S.q_full[slot], (uint32_t)(qi / kQueue) & 1u, S, args.status);
       if (!__all_sync(0xffffffffu, got)) break;
@@ -401,17 +433,18 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       if (tile < 0) break;
       const Geom G = tile_geom<MODE>(args, S, tile, R);
       const Tile& tl = G.t;
-      const int buf = tcount & 1;
-      const uint32_t use = (uint32_t)(tcount >> 1) & 1u;
-      const uint32_t base = tmem + lane_off + buf * kBufCols;
-      // down: token and weight of columns lane, lane + 32, ... requested before waiting for
-      // the accumulators, so the loads overlap the tile's MMAs
-      int col_tok[kColChunks];
-      float col_w[kColChunks];
+      int first, count;
+      sl.take(tl.N, first, count);
+      const uint32_t b0 = tmem + lane_off + first * kSlotCols;
+      const uint32_t b1 = b0 + (count == 2 ? kSlotCols : 128u);
+      // down: token and weight of this warp's columns, requested before waiting for the
+      // accumulators so that the loads overlap the tile's MMAs
+      int col_tok[kChunks];
+      float col_w[kChunks];
       if (MODE == kDown) {
 #pragma unroll
-        for (int ci = 0; ci < kColChunks; ++ci) {
-          const int c = ci * 32 + lane;
+        for (int ci = 0; ci < kChunks; ++ci) {
+          const int c = (2 * ci + half) * 32 + lane;
           col_tok[ci] = 0;
           col_w[ci] = 0.f;
           if (c < tl.nvalid) {
@@ -421,16 +454,20 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           }
         }
       }
-      const bool ok = wait_phase(&S.tmem_full[buf], use, S, args.status);
+      bool ok = true;
+      for (int i = 0; i < count; ++i) {
+        const int sidx = (first + i) & 1;
+        ok = ok && wait_phase(&S.tmem_full[sidx], sl.uses[sidx] & 1u, S, args.status);
+      }
       if (!__all_sync(0xffffffffu, ok)) break;
       ptx::tc_fence_after();
 #pragma unroll
-      for (int ci = 0; ci < kColChunks; ++ci) {
-        const int c0 = ci * 32;
+      for (int ci = 0; ci < kChunks; ++ci) {
+        const int c0 = (2 * ci + half) * 32;
         if (c0 >= tl.nvalid) break;
         uint32_t r0[32], r1[32];
-        ptx::tmem_ld32(base + c0, r0);
-        ptx::tmem_ld32(base + 128 + c0, r1);
+        ptx::tmem_ld32(b0 + c0, r0);
+        ptx::tmem_ld32(b1 + c0, r1);
         ptx::tmem_ld_wait();
         if (MODE == kGateUp) {
           const int ch = tl.m * 128 + qd * 32 + lane;
@@ -485,7 +522,8 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         }
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&S.tmem_empty[buf]);
+      for (int i = 0; i < count; ++i) ptx::mbar_arrive(&S.tmem_empty[(first + i) & 1]);
+      sl.done(first, count);
     }
   }
 
@@ -557,8 +595,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer][inner] (inner contiguous), box [box_outer][box_inner],
-// 128-byte swizzle (box_inner = 64 elements = 128 bytes).
+// 2-D bf16 tensor [outer][inner] (inner contiguous), box [box_outer][box_inner] with the
+// swizzle matching box_inner (64 elements: 128-byte swizzle, 32: 64-byte swizzle).
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
               uint32_t box_inner, uint32_t box_outer) {
   auto fn = encode_fn();
@@ -567,9 +605,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
   cuuint64_t strides[1] = {inner * sizeof(uint16_t)};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw =
+      box_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int sm_count() {
@@ -621,6 +661,7 @@ bool tc_router_supported(const moe_shape& s) {
 
 cudaError_t launch_tc_router(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                              const float* wr, float* logits, cudaStream_t st) {
+  using C = Cfg<kRouter>;
   uint16_t* split = reinterpret_cast<uint16_t*>(ws + L.wr_split);
   {
     LaunchScope scope(MOE_K_OTHER, st);
@@ -632,13 +673,13 @@ cudaError_t launch_tc_router(const moe_shape& s, const Layout& L, char* ws, cons
     if (e != cudaSuccess) return e;
   }
   CUtensorMap a, b;
-  if (!make_map(&a, split, 3ull * s.H, (uint64_t)s.E, 64, 128) ||
-      !make_map(&b, x, s.H, (uint64_t)s.T, 64, kBoxRows))
+  if (!make_map(&a, split, 3ull * s.H, (uint64_t)s.E, C::kBK, 128) ||
+      !make_map(&b, x, s.H, (uint64_t)s.T, C::kBK, kBoxRows))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.logits = logits;
+  args.ntiles = ((s.E + 255) / 256) * ((s.T + C::kMaxTile - 1) / C::kMaxTile);
   args.counter = reinterpret_cast<int*>(ws + L.sched) + 2;
-  args.ntiles = ((s.E + 255) / 256) * ((s.T + kMaxTile - 1) / kMaxTile);
   LaunchScope scope(MOE_K_ROUTER_LOGITS, st);
   return launch_mode<kRouter>(a, a, b, b, args, std::min(args.ntiles, sm_count()), st);
 }
@@ -650,6 +691,7 @@ bool tc_supported(const moe_shape& s) {
 
 cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                               const int32_t* sorted_token, const moe_weights& w, cudaStream_t st) {
+  using C = Cfg<kGateUp>;
   uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
   {
     LaunchScope scope(MOE_K_OTHER, st);
@@ -660,10 +702,10 @@ cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, con
     if (e != cudaSuccess) return e;
   }
   CUtensorMap a, a_sh, b, b_sh;
-  if (!make_map(&a, w.w_gate_up, s.H, (uint64_t)s.E * 2 * s.I, 64, 128) ||
-      !make_map(&a_sh, w.ws_gate_up, s.H, 2ull * s.Is, 64, 128) ||
-      !make_map(&b, xs, s.H, (uint64_t)s.T * s.k, 64, kBoxRows) ||
-      !make_map(&b_sh, x, s.H, (uint64_t)s.T, 64, kBoxRows))
+  if (!make_map(&a, w.w_gate_up, s.H, (uint64_t)s.E * 2 * s.I, C::kBK, 128) ||
+      !make_map(&a_sh, w.ws_gate_up, s.H, 2ull * s.Is, C::kBK, 128) ||
+      !make_map(&b, xs, s.H, (uint64_t)s.T * s.k, C::kBK, kBoxRows) ||
+      !make_map(&b_sh, x, s.H, (uint64_t)s.T, C::kBK, kBoxRows))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
@@ -677,10 +719,11 @@ cudaError_t launch_tc_down(const moe_shape& s, const Layout& L, char* ws,
                            const int32_t* sorted_token, const float* sorted_w, const float* sgate,
                            const moe_weights& w, float* y, float* y_shared, float* out,
                            cudaStream_t st) {
+  using C = Cfg<kDown>;
   CUtensorMap a, a_sh, b;
-  if (!make_map(&a, w.w_down, s.I, (uint64_t)s.E * s.H, 64, 128) ||
-      !make_map(&a_sh, w.ws_down, s.Is, (uint64_t)s.H, 64, 128) ||
-      !make_map(&b, ws + L.h, L.ldh, 2 * (L.h_plane / L.ldh), 64, kBoxRows))
+  if (!make_map(&a, w.w_down, s.I, (uint64_t)s.E * s.H, C::kBK, 128) ||
+      !make_map(&a_sh, w.ws_down, s.Is, (uint64_t)s.H, C::kBK, 128) ||
+      !make_map(&b, ws + L.h, L.ldh, 2 * (L.h_plane / L.ldh), C::kBK, kBoxRows))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
