@@ -72,8 +72,8 @@ __host__ __device__ inline PlanView plan_view(void* base, int E) {
 }
 
 // Tensor-core tiling of a group with n rows into ceil(n / max) token chunks of nearly equal
-// size (multiples of 16 rows), max 256 rows for both grouped GEMMs.
-constexpr int kTcChunkDown = kTcChunk;
+// size (multiples of 16 rows): max 256 rows for the gate|up GEMM, 128 for the down GEMM.
+constexpr int kTcChunkDown = 128;
 __host__ __device__ inline int tc_nchunks(int n, int max_rows) {
   return (n + max_rows - 1) / max_rows;
 }

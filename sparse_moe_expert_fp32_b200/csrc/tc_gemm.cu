@@ -5,17 +5,16 @@
 //
 // Orientation ("swap AB"): weight rows are the MMA's M side (two 128-row accumulators per
 // tile = 256 weight rows sharing one token tile), the tokens of one expert are the N side
-// (multiples of 16, up to 256 per tile, so a prefill expert is one tile and its weights
-// pass through shared memory once), K is the hidden (gate|up, router) or intermediate
-// (down) dimension.
+// (multiples of 16; up to 256 per gate|up tile, so a prefill expert is one tile and its
+// gate|up weights pass through shared memory once; up to 128 per down and router tile),
+// K is the hidden (gate|up, router) or intermediate (down) dimension.
 //
 //   gate|up: gate rows [c, c+128) and up rows [I+c, I+c+128) of one expert against its
 //     token rows, copied beforehand in dispatch order (gather_rows_kernel) so that a token
 //     tile is a few plain 2-D TMA boxes. Epilogue: h = SiLU(gate) * up stored as the bf16
 //     pair hi = bf16(h), lo = bf16(h - hi).
 //   down: 256 rows of one expert's W_down against its packed rows; per K step two MMAs add
-//     W h_hi and W h_lo into the same accumulators (32-wide K stages, 64-byte swizzle, so
-//     that a 256-token tile still leaves four stages). Epilogue: y rows (staged path) or
+//     W h_hi and W h_lo into the same accumulators. Epilogue: y rows (staged path) or
 //     routing-weight-scaled fp32 atomic adds into out[token] ("Weighted combine + gated
 //     shared expert").
 //   router: 256 experts x 128 tokens of logits = x . (hi + mid + lo)^T, K = 3H over the
@@ -56,17 +55,19 @@ constexpr int kQueue = 4;  // tile ids handed from the producer to the MMA and e
 
 enum Mode { kGateUp = 0, kDown = 1, kRouter = 2 };
 
-// Per-mode pipeline geometry.
+// Per-mode pipeline geometry. The down GEMM keeps tiles of at most 128 tokens: its K loop
+// is short (K = I), so its epilogue must overlap the next tile's MMAs (one TMEM slot per
+// tile); a 256-token down tile measured 1.36x slower on the Flash-Next prefill layer.
 template <int MODE>
 struct Cfg {
-  static constexpr int kBK = (MODE == kDown) ? 32 : 64;        // K per stage
-  static constexpr int kRowBytes = kBK * 2;                      // 64 or 128 (= swizzle)
-  static constexpr int kMaxTile = (MODE == kRouter) ? 128 : 256;  // tokens per tile
+  static constexpr int kBK = 64;                                  // K per stage
+  static constexpr int kRowBytes = kBK * 2;                       // 128 (= swizzle)
+  static constexpr int kMaxTile = (MODE == kGateUp) ? 256 : 128;  // tokens per tile
   static constexpr uint32_t kATileBytes = 128u * kRowBytes;
   static constexpr uint32_t kBTileBytes = (uint32_t)kMaxTile * kRowBytes;
   static constexpr int kBTiles = (MODE == kDown) ? 2 : 1;  // down: hi and lo rows of h
   static constexpr uint32_t kStageBytes = 2 * kATileBytes + kBTiles * kBTileBytes;
-  static constexpr int kStages = (MODE == kDown) ? 4 : 3;
+  static constexpr int kStages = 3;
   static constexpr int kKK = kBK / 16;  // MMAs (K = 16) per stage and accumulator
 };
 
@@ -83,12 +84,16 @@ struct SharedState {
   int q[kQueue];
   int tp[kMaxE + 2];    // tile prefix of the grouped GEMM (copied from the plan)
   int row0[kMaxE + 2];  // first packed row of each group (copied from the plan)
+  float4 xpose[kEpiWarps][8][8];  // down epilogue: per warp, 8 tokens x 32 channels
 };
 
 template <int MODE>
 constexpr size_t smem_bytes() {
   return 1024 + (size_t)Cfg<MODE>::kStages * Cfg<MODE>::kStageBytes + sizeof(SharedState);
 }
+static_assert(smem_bytes<kGateUp>() <= 232448 && smem_bytes<kDown>() <= 232448 &&
+                  smem_bytes<kRouter>() <= 232448,
+              "over the 227 KB of shared memory a CTA may use");
 
 struct TcArgs {
   const int* plan;
@@ -495,27 +500,40 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             }
           }
         } else {
-          const int m = tl.m * 256 + qd * 32 + lane;  // rows m (first accumulator), m + 128
+          // 32 channels (lanes) x 32 tokens (registers) per accumulator; every 8 tokens go
+          // through shared memory so that a lane owns 8 consecutive channels of one token
+          // and writes them with two 16-byte stores or atomic adds
+          const int mrow = tl.m * 256 + qd * 32 + 8 * (lane & 3);  // this lane's channels
           const int H = args.H;
+          float4(&xp)[8][8] = S.xpose[warp - 2];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (c0 + j < tl.nvalid) {
-              const float y0 = __uint_as_float(r0[j]), y1 = __uint_as_float(r1[j]);
-              const int t = __shfl_sync(0xffffffffu, col_tok[ci], j);
-              const float w = __shfl_sync(0xffffffffu, col_w[ci], j);
-              const int p = tl.p0 + c0 + j;
-              if (args.out) {
-                float* o = args.out + (size_t)t * H + m;
-                atomicAdd(o, w * y0);
-                atomicAdd(o + 128, w * y1);
-              } else if (p < R) {
-                float* o = args.y + (size_t)p * H + m;
-                o[0] = y0;
-                o[128] = y1;
-              } else {
-                float* o = args.y_shared + (size_t)(p - R) * H + m;
-                o[0] = y0;
-                o[128] = y1;
+          for (int acc = 0; acc < 2; ++acc) {
+            const uint32_t* r = acc ? r1 : r0;
+#pragma unroll
+            for (int sb = 0; sb < 4; ++sb) {
+              __syncwarp();
+              float* xs = reinterpret_cast<float*>(&xp[0][0]);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) xs[q * 32 + lane] = __uint_as_float(r[sb * 8 + q]);
+              __syncwarp();
+              const int q = lane >> 2;  // this lane's token within the 8
+              const float4 v0 = xp[q][2 * (lane & 3)], v1 = xp[q][2 * (lane & 3) + 1];
+              const int col = c0 + sb * 8 + q;
+              const int t = __shfl_sync(0xffffffffu, col_tok[ci], sb * 8 + q);
+              const float w = __shfl_sync(0xffffffffu, col_w[ci], sb * 8 + q);
+              if (col < tl.nvalid) {
+                const int p = tl.p0 + col;
+                const int m = mrow + acc * 128;
+                if (args.out) {
+                  float4* o = reinterpret_cast<float4*>(args.out + (size_t)t * H + m);
+                  atomicAdd(o, make_float4(w * v0.x, w * v0.y, w * v0.z, w * v0.w));
+                  atomicAdd(o + 1, make_float4(w * v1.x, w * v1.y, w * v1.z, w * v1.w));
+                } else {
+                  float* row = p < R ? args.y + (size_t)p * H : args.y_shared + (size_t)(p - R) * H;
+                  float4* o = reinterpret_cast<float4*>(row + m);
+                  o[0] = v0;
+                  o[1] = v1;
+                }
               }
             }
           }
