@@ -22,7 +22,8 @@
 //
 // Roles in a 320-thread CTA (one CTA per SM, persistent; tiles handed out in order by an
 // atomic counter through a shared-memory queue):
-//   warp 0      TMA producer (lane 0 issues) over a ring of kStages stages;
+//   warp 0      TMA producer over a ring of kStages stages (lane 0 takes tiles and arms
+//               the barriers; each box of a stage is issued by its own lane);
 //   warp 1      TMEM owner (all 512 columns, two slots of 256) and MMA issuer (lane 0);
 //               a tile of at most 128 tokens takes one slot (its two accumulators are
 //               128 columns each) and the next tile's MMAs fill the other slot while the
@@ -46,7 +47,12 @@ namespace {
 
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kBoxRows = 16;  // rows per TMA box of a token tile
+// A token tile of N rows (a multiple of 16) is loaded as at most five TMA boxes of 128, 64,
+// 32 or 16 rows (128-row boxes first, then the binary digits of the rest): a TMA
+// instruction costs about as much as moving 60-70 rows, so sixteen-row boxes alone made
+// the token loads the slowest part of a prefill stage.
+constexpr int kBoxHeights = 4;
+__host__ __device__ constexpr int box_rows_of(int i) { return 128 >> i; }
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 constexpr uint32_t kTmemCols = 512;
@@ -94,6 +100,37 @@ constexpr size_t smem_bytes() {
 static_assert(smem_bytes<kGateUp>() <= 232448 && smem_bytes<kDown>() <= 232448 &&
                   smem_bytes<kRouter>() <= 232448,
               "over the 227 KB of shared memory a CTA may use");
+
+// The token operand's tensor map in each box height (index i: 128 >> i rows).
+struct BMaps {
+  CUtensorMap m[kBoxHeights];
+};
+
+// Piece `j` of an N-row token tile: its first row and box-height index; false past the
+// last piece.
+__device__ __forceinline__ bool token_piece(int N, int j, int& row, int& hidx) {
+  const int n128 = N >> 7;
+  if (j < n128) {
+    row = j * 128;
+    hidx = 0;
+    return true;
+  }
+  j -= n128;
+  int r = n128 * 128;
+#pragma unroll
+  for (int h = 1; h < kBoxHeights; ++h) {
+    if (N & box_rows_of(h)) {
+      if (j == 0) {
+        row = r;
+        hidx = h;
+        return true;
+      }
+      --j;
+      r += box_rows_of(h);
+    }
+  }
+  return false;
+}
 
 struct TcArgs {
   const int* plan;
@@ -246,7 +283,7 @@ struct Slots {
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_sh,
-                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b_sh,
+                  const __grid_constant__ BMaps tm_b, const __grid_constant__ BMaps tm_b_sh,
                   const TcArgs args) {
   using C = Cfg<MODE>;
   extern __shared__ uint8_t smem_raw[];
@@ -289,8 +326,10 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tm_a);
     ptx::prefetch_tmap(&tm_a_sh);
-    ptx::prefetch_tmap(&tm_b);
-    ptx::prefetch_tmap(&tm_b_sh);
+    for (int i = 0; i < kBoxHeights; ++i) {
+      ptx::prefetch_tmap(&tm_b.m[i]);
+      ptx::prefetch_tmap(&tm_b_sh.m[i]);
+    }
   }
   if (warp == 1) {
     ptx::tmem_alloc(&S.tmem_base, kTmemCols);
@@ -303,58 +342,82 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int it = 0;
-      int armed[C::kStages];
+    // Lane 0 takes tiles, waits for free stages and arms the full barriers; then every
+    // lane with a box of the stage issues it (lanes 0-1: the two weight boxes, lanes 2..:
+    // the token pieces, hi plane then lo plane for down), so the copies start together.
+    int it = 0;
+    int armed[C::kStages];
 #pragma unroll
-      for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
-      bool aborted = false;
-      const int plane_rows = (MODE == kDown) ? (int)(args.h_plane / (size_t)args.ldh) : 0;
-      // tiles are handed out in order by one counter: neighbouring tiles (the chunks of one
-      // weight tile, the M tiles of one expert) run at the same time on neighbouring SMs
-      for (int qi = 0; !aborted; ++qi) {
-        const int slot = qi % kQueue;
+    for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
+    bool aborted = false;
+    const int plane_rows = (MODE == kDown) ? (int)(args.h_plane / (size_t)args.ldh) : 0;
+    // tiles are handed out in order by one counter: neighbouring tiles (the chunks of one
+    // weight tile, the M tiles of one expert) run at the same time on neighbouring SMs
+    for (int qi = 0; !aborted; ++qi) {
+      const int slot = qi % kQueue;
+      int tile = 0;
+      if (lane == 0) {
         if (!wait_phase(&S.q_empty[slot], ((uint32_t)(qi / kQueue) & 1u) ^ 1u, S, args.status)) {
+          tile = -2;
+        } else {
+          tile = atomicAdd(args.counter, 1);
+          if (tile >= total) tile = -1;
+          S.q[slot] = tile;
+          ptx::mbar_arrive(&S.q_full[slot]);
+        }
+      }
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      if (tile == -2) aborted = true;
+      if (tile < 0) break;
+      const Geom G = tile_geom<MODE>(args, S, tile, R);
+      // this lane's box: weight rows (lanes 0, 1) or one token piece of one plane
+      const CUtensorMap* my_map = nullptr;
+      uint32_t my_off = 0;
+      int my_row = 0;
+      if (lane < 2) {
+        my_map = G.shared ? &tm_a_sh : &tm_a;
+        my_off = lane * C::kATileBytes;
+        my_row = lane ? G.a_row1 : G.a_row0;
+      } else {
+        int np = 0, r, h;
+        while (token_piece(G.t.N, np, r, h)) ++np;
+        const int j = lane - 2;
+        if (j < np * C::kBTiles) {
+          const int plane = j / np;
+          token_piece(G.t.N, j - plane * np, r, h);
+          const BMaps& bm = (MODE == kGateUp && G.shared) ? tm_b_sh : tm_b;
+          my_map = &bm.m[h];
+          my_off = 2 * C::kATileBytes + plane * C::kBTileBytes + (uint32_t)r * C::kRowBytes;
+          my_row = G.b_row0 + r + plane * plane_rows;
+        }
+      }
+      const uint32_t bytes = 2 * C::kATileBytes + (uint32_t)C::kBTiles * G.t.N * C::kRowBytes;
+      for (int ks = 0; ks < G.nk; ++ks, ++it) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+        bool ok = true;
+        if (lane == 0) {
+          ok = wait_phase(&S.empty[s], ph ^ 1u, S, args.status);
+          if (ok) {
+            ptx::mbar_arrive_expect_tx(&S.full[s], bytes);
+            armed[s] = (int)ph;
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
           aborted = true;
           break;
         }
-        int tile = atomicAdd(args.counter, 1);
-        if (tile >= total) tile = -1;
-        S.q[slot] = tile;
-        ptx::mbar_arrive(&S.q_full[slot]);
-        if (tile < 0) break;
-        const Geom G = tile_geom<MODE>(args, S, tile, R);
-        const CUtensorMap* ta = G.shared ? &tm_a_sh : &tm_a;
-        const CUtensorMap* tb = (MODE == kGateUp && G.shared) ? &tm_b_sh : &tm_b;
-        const uint32_t bytes = 2 * C::kATileBytes + (uint32_t)C::kBTiles * G.t.N * C::kRowBytes;
-        for (int ks = 0; ks < G.nk; ++ks, ++it) {
-          const int s = it % C::kStages;
-          const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
-          if (!wait_phase(&S.empty[s], ph ^ 1u, S, args.status)) {
-            aborted = true;
-            break;
-          }
-          ptx::mbar_arrive_expect_tx(&S.full[s], bytes);
-          armed[s] = (int)ph;
-          uint8_t* st = smem + s * C::kStageBytes;
+        if (my_map) {
           const int ka = ks * C::kBK;
-          ptx::tma_load_2d(st, ta, &S.full[s], ka, G.a_row0);
-          ptx::tma_load_2d(st + C::kATileBytes, ta, &S.full[s], ka, G.a_row1);
-          uint8_t* b = st + 2 * C::kATileBytes;
-          const int kx = (MODE == kRouter) ? ka % args.H : ka;
-          for (int j = 0; j < G.t.N; j += kBoxRows) {
-            ptx::tma_load_2d(b + j * C::kRowBytes, tb, &S.full[s], kx, G.b_row0 + j);
-            if (MODE == kDown)
-              ptx::tma_load_2d(b + C::kBTileBytes + j * C::kRowBytes, tb, &S.full[s], kx,
-                               plane_rows + G.b_row0 + j);
-          }
+          const int kx = (MODE == kRouter && lane >= 2) ? ka % args.H : ka;
+          ptx::tma_load_2d(smem + s * C::kStageBytes + my_off, my_map, &S.full[s], kx, my_row);
         }
       }
-      if (aborted) {
-        // let this CTA's copies in flight land before the shared memory is released
-        for (int s = 0; s < C::kStages; ++s)
-          if (armed[s] >= 0) drain_phase(&S.full[s], (uint32_t)armed[s]);
-      }
+    }
+    if (aborted && lane == 0) {
+      // let this CTA's copies in flight land before the shared memory is released
+      for (int s = 0; s < C::kStages; ++s)
+        if (armed[s] >= 0) drain_phase(&S.full[s], (uint32_t)armed[s]);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -630,6 +693,13 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The token tensor [outer][inner] in every box height of a token tile.
+bool make_bmaps(BMaps* b, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner) {
+  for (int i = 0; i < kBoxHeights; ++i)
+    if (!make_map(&b->m[i], base, inner, outer, box_inner, (uint32_t)box_rows_of(i))) return false;
+  return true;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   cudaGetDevice(&dev);
@@ -638,8 +708,8 @@ int sm_count() {
 }
 
 template <int MODE>
-cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& a_sh, const CUtensorMap& b,
-                        const CUtensorMap& b_sh, const TcArgs& args, int grid, cudaStream_t st) {
+cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& a_sh, const BMaps& b,
+                        const BMaps& b_sh, const TcArgs& args, int grid, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -690,9 +760,10 @@ cudaError_t launch_tc_router(const moe_shape& s, const Layout& L, char* ws, cons
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap a, b;
+  CUtensorMap a;
+  BMaps b;
   if (!make_map(&a, split, 3ull * s.H, (uint64_t)s.E, C::kBK, 128) ||
-      !make_map(&b, x, s.H, (uint64_t)s.T, C::kBK, kBoxRows))
+      !make_bmaps(&b, x, s.H, (uint64_t)s.T, C::kBK))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.logits = logits;
@@ -719,11 +790,12 @@ cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, con
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap a, a_sh, b, b_sh;
+  CUtensorMap a, a_sh;
+  BMaps b, b_sh;
   if (!make_map(&a, w.w_gate_up, s.H, (uint64_t)s.E * 2 * s.I, C::kBK, 128) ||
       !make_map(&a_sh, w.ws_gate_up, s.H, 2ull * s.Is, C::kBK, 128) ||
-      !make_map(&b, xs, s.H, (uint64_t)s.T * s.k, C::kBK, kBoxRows) ||
-      !make_map(&b_sh, x, s.H, (uint64_t)s.T, C::kBK, kBoxRows))
+      !make_bmaps(&b, xs, s.H, (uint64_t)s.T * s.k, C::kBK) ||
+      !make_bmaps(&b_sh, x, s.H, (uint64_t)s.T, C::kBK))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
@@ -738,10 +810,11 @@ cudaError_t launch_tc_down(const moe_shape& s, const Layout& L, char* ws,
                            const moe_weights& w, float* y, float* y_shared, float* out,
                            cudaStream_t st) {
   using C = Cfg<kDown>;
-  CUtensorMap a, a_sh, b;
+  CUtensorMap a, a_sh;
+  BMaps b;
   if (!make_map(&a, w.w_down, s.I, (uint64_t)s.E * s.H, C::kBK, 128) ||
       !make_map(&a_sh, w.ws_down, s.Is, (uint64_t)s.H, C::kBK, 128) ||
-      !make_map(&b, ws + L.h, L.ldh, 2 * (L.h_plane / L.ldh), C::kBK, kBoxRows))
+      !make_bmaps(&b, ws + L.h, L.ldh, 2 * (L.h_plane / L.ldh), C::kBK))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
