@@ -564,9 +564,11 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           }
         } else {
           // 32 channels (lanes) x 32 tokens (registers) per accumulator; every 8 tokens go
-          // through shared memory so that a lane owns 8 consecutive channels of one token
-          // and writes them with two 16-byte stores or atomic adds
-          const int mrow = tl.m * 256 + qd * 32 + 8 * (lane & 3);  // this lane's channels
+          // through shared memory so that eight lanes own the 32 channels (128 bytes) of one
+          // token, four tokens per instruction: every 16-byte atomic add or store of a
+          // warp lands in whole 128-byte lines (a lane-per-channel order, or two 16-byte
+          // pieces 32 bytes apart, cut the reduction throughput by a third)
+          const int mrow = tl.m * 256 + qd * 32 + 4 * (lane & 7);  // this lane's channels
           const int H = args.H;
           float4(&xp)[8][8] = S.xpose[warp - 2];
 #pragma unroll
@@ -579,23 +581,24 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 #pragma unroll
               for (int q = 0; q < 8; ++q) xs[q * 32 + lane] = __uint_as_float(r[sb * 8 + q]);
               __syncwarp();
-              const int q = lane >> 2;  // this lane's token within the 8
-              const float4 v0 = xp[q][2 * (lane & 3)], v1 = xp[q][2 * (lane & 3) + 1];
-              const int col = c0 + sb * 8 + q;
-              const int t = __shfl_sync(0xffffffffu, col_tok[ci], sb * 8 + q);
-              const float w = __shfl_sync(0xffffffffu, col_w[ci], sb * 8 + q);
-              if (col < tl.nvalid) {
-                const int p = tl.p0 + col;
-                const int m = mrow + acc * 128;
-                if (args.out) {
-                  float4* o = reinterpret_cast<float4*>(args.out + (size_t)t * H + m);
-                  atomicAdd(o, make_float4(w * v0.x, w * v0.y, w * v0.z, w * v0.w));
-                  atomicAdd(o + 1, make_float4(w * v1.x, w * v1.y, w * v1.z, w * v1.w));
-                } else {
-                  float* row = p < R ? args.y + (size_t)p * H : args.y_shared + (size_t)(p - R) * H;
-                  float4* o = reinterpret_cast<float4*>(row + m);
-                  o[0] = v0;
-                  o[1] = v1;
+#pragma unroll
+              for (int hq = 0; hq < 2; ++hq) {
+                const int q = hq * 4 + (lane >> 3);  // this lane's token within the 8
+                const float4 v = xp[q][lane & 7];
+                const int col = c0 + sb * 8 + q;
+                const int t = __shfl_sync(0xffffffffu, col_tok[ci], sb * 8 + q);
+                const float w = __shfl_sync(0xffffffffu, col_w[ci], sb * 8 + q);
+                if (col < tl.nvalid) {
+                  const int p = tl.p0 + col;
+                  const int m = mrow + acc * 128;
+                  if (args.out) {
+                    atomicAdd(reinterpret_cast<float4*>(args.out + (size_t)t * H + m),
+                              make_float4(w * v.x, w * v.y, w * v.z, w * v.w));
+                  } else {
+                    float* row =
+                        p < R ? args.y + (size_t)p * H : args.y_shared + (size_t)(p - R) * H;
+                    *reinterpret_cast<float4*>(row + m) = v;
+                  }
                 }
               }
             }
