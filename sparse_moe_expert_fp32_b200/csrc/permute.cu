@@ -12,6 +12,8 @@
 //                           its expert plus the number of earlier tokens of the block in
 //                           the same mask -- token-ascending inside each expert, and the
 //                           same on every run.
+// With T <= 256 (one token block, e.g. decode) dispatch_small_kernel does all three steps in
+// one CTA with the masks in shared memory; the result is the same.
 // An expert id outside [0, E) is skipped and raises the bounds flag in the status word.
 #include <mutex>
 
@@ -184,6 +186,69 @@ dispatch_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict
   }
 }
 
+// The three steps above for T <= kPermBlock in one CTA of kScanThreads threads: thread
+// i < T marks token i in the shared-memory masks, thread e < E counts and scans expert e
+// (offsets, plan), then token i places its k assignments.
+__global__ void __launch_bounds__(kScanThreads)
+dispatch_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int T,
+                      int E, int k, int H, int I, int Is, int32_t* __restrict__ offsets,
+                      int* __restrict__ plan_base, int32_t* __restrict__ sorted_token,
+                      float* __restrict__ sorted_w, int32_t* __restrict__ assign_row,
+                      uint32_t* __restrict__ status) {
+  extern __shared__ uint32_t mask[];  // [E][8]
+  __shared__ int smem[33];
+  __shared__ int n_of[kMaxE + 1];
+  __shared__ int base[kMaxE];
+  for (int q = threadIdx.x; q < E * 8; q += blockDim.x) mask[q] = 0;
+  __syncthreads();
+  const int i = threadIdx.x;
+  if (i < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[(size_t)i * k + j];
+      if (e < 0 || e >= E) {
+        set_flag(status, kFlagBounds);
+        continue;
+      }
+      atomicOr(&mask[e * 8 + (i >> 5)], 1u << (i & 31));
+    }
+  }
+  __syncthreads();
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) total += __popc(mask[e * 8 + w]);
+  }
+  int R;
+  const int off = block_exclusive_scan(e < E ? total : 0, smem, &R);
+  if (e < E) {
+    offsets[e] = off;
+    base[e] = off;
+    n_of[e] = total;
+  }
+  if (threadIdx.x == 0) {
+    offsets[E] = R;
+    n_of[E] = T;
+  }
+  __syncthreads();
+  build_plan(n_of, E, H, I, Is, plan_view(plan_base, E), smem);
+  if (i < T) {
+    const int word = i >> 5;
+    const uint32_t below = (1u << (i & 31)) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int ee = ids[(size_t)i * k + j];
+      if (ee < 0 || ee >= E) continue;
+      const uint32_t* m = mask + ee * 8;
+      int rank = __popc(m[word] & below);
+      for (int w = 0; w < word; ++w) rank += __popc(m[w]);
+      const int p = base[ee] + rank;
+      sorted_token[p] = i;
+      if (sorted_w) sorted_w[p] = topk_w[(size_t)i * k + j];
+      assign_row[(size_t)i * k + j] = p;
+    }
+  }
+}
+
 // Plan from caller-supplied offsets. Offsets that are not a monotone partition of at most
 // T*k rows starting at 0 are flagged and give an empty plan (no GEMM work).
 __global__ void __launch_bounds__(kScanThreads)
@@ -214,11 +279,18 @@ plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int T, int E, int 
 cudaError_t launch_permute(const moe_shape& s, const Layout& L, char* ws, const int32_t* ids,
                            const float* topk_w, int32_t* offsets, int32_t* sorted_token,
                            float* sorted_w, int32_t* assign_row, cudaStream_t st) {
-  LaunchScope scope(MOE_K_PERMUTE, st, 3);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
   uint32_t* blk_mask = reinterpret_cast<uint32_t*>(ws + L.blk_mask);
   int32_t* blk_base = reinterpret_cast<int32_t*>(ws + L.blk_base);
   const size_t smem = (size_t)s.E * 8 * sizeof(uint32_t);
+  if (s.T <= kPermBlock) {
+    LaunchScope scope(MOE_K_PERMUTE, st);
+    dispatch_small_kernel<<<1, kScanThreads, smem, st>>>(
+        ids, topk_w, s.T, s.E, s.k, s.H, s.I, s.Is, offsets, reinterpret_cast<int*>(ws + L.plan),
+        sorted_token, sorted_w, assign_row, status);
+    return cudaGetLastError();
+  }
+  LaunchScope scope(MOE_K_PERMUTE, st, 3);
   // counts go to blk_base first, the scan rewrites them in place as bases
   dispatch_mask_kernel<<<L.nblk, kPermBlock, smem, st>>>(ids, s.T, s.E, s.k, blk_mask, blk_base,
                                                         status);

@@ -6,10 +6,14 @@
 //   router_logits_small_kernel  : logits = x . Wr^T on CUDA cores for small batches, as
 //                                 four partial sums over hidden-dimension slices; larger
 //                                 batches use the tensor-core router in tc_gemm.cu.
-//   router_topk_kernel          : one warp per token: top-k with lowest-index ties,
-//                                 renormalised softmax weights, 10th/11th gap,
-//                                 shared-expert gate sigmoid(w_shared . x).
+//   router_topk_kernel          : two warps per token: one takes the top-k with
+//                                 lowest-index ties, the renormalised softmax weights and
+//                                 the 10th/11th gap, the other the shared-expert gate
+//                                 sigmoid(w_shared . x) and the zeroing of the token's
+//                                 output row.
 #include <float.h>
+
+#include <mutex>
 
 #include "device_common.cuh"
 #include "moe_internal.h"
@@ -20,21 +24,29 @@ namespace {
 
 // Small batches (T < 512): partial logits over kSplits slices of the hidden dimension,
 // part[s][t][e] = sum_{h in slice s} x[t][h] * wr[e][h], fp32 FMAs in h order. A CTA
-// computes 16 experts x 64 tokens of one slice: x and wr chunks are staged in shared
-// memory (x transposed so that a warp's 32 tokens read consecutive words), each thread
-// accumulates 4 experts x 1 token. The top-k kernel adds the slices in order s = 0..3, so
-// the logits are the same on every run. Grid (ceil(E/16), kSplits, ceil(T/64)) fills the
-// GPU at decode sizes (128 CTAs at E = 512, T = 64) and reads wr once.
+// computes 16 experts x 64 tokens of one slice: x and wr chunks of 128 hidden positions are
+// staged in shared memory (x transposed so that a warp's 32 tokens read consecutive words),
+// double-buffered -- the next chunk's global loads are in flight while the current one is
+// multiplied -- and each thread accumulates 4 experts x 1 token. The top-k kernel adds the
+// slices in order s = 0..3, so the logits are the same on every run. Grid
+// (ceil(E/16), kSplits, ceil(T/64)) fills the GPU at decode sizes (128 CTAs at E = 512,
+// T = 64) and reads wr once.
 constexpr int kSplits = 4;
 constexpr int kSmallTok = 64;
 constexpr int kSmallExp = 16;
 constexpr int kSmallKc = 128;
+constexpr int kSmallThreads = 256;
+constexpr int kSmallXLoads = kSmallTok * (kSmallKc / 8) / kSmallThreads;  // uint4 per thread
+constexpr int kSmallWLoads = kSmallExp * (kSmallKc / 4) / kSmallThreads;  // float4 per thread
+constexpr size_t kSmallSmem =
+    2 * (size_t)kSmallKc * kSmallTok * sizeof(float) + 2 * (size_t)kSmallKc * kSmallExp * sizeof(float);
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kSmallThreads)
 router_logits_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
                            float* __restrict__ part, int T, int H, int E, int nslices) {
-  __shared__ float xs[kSmallKc][kSmallTok];
-  __shared__ float4 wsm[kSmallKc][kSmallExp / 4];
+  extern __shared__ float4 dsm[];
+  float* xs_all = reinterpret_cast<float*>(dsm);                            // [2][Kc][Tok]
+  float* ws_all = xs_all + 2 * kSmallKc * kSmallTok;                       // [2][Kc][Exp]
   const int e0 = blockIdx.x * kSmallExp;
   const int t0 = blockIdx.z * kSmallTok;
   const int slice = H / nslices;  // a multiple of 16 (H is a multiple of 64)
@@ -42,37 +54,72 @@ router_logits_small_kernel(const uint16_t* __restrict__ x, const float* __restri
   const int tid = threadIdx.x;
   const int tok = tid & (kSmallTok - 1), eg = tid >> 6;  // 4 expert groups of 4
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  uint4 xr[kSmallXLoads];
+  float4 wv[kSmallWLoads];
 
-  for (int k0 = kbeg; k0 < kend; k0 += kSmallKc) {
-    const int kn = min(kSmallKc, kend - k0);  // multiple of 16
-    const int x8 = kn / 8;
-    for (int i = tid; i < kSmallTok * x8; i += blockDim.x) {
-      const int r = i % kSmallTok, c = i / kSmallTok;  // consecutive threads: consecutive tokens
-      float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (t0 + r < T) unpack8(ld_v4(x + (size_t)(t0 + r) * H + k0 + 8 * c), f);
+  // global -> registers for the chunk at k0 (zeros outside the tensor)
+  auto load = [&](int k0) {
+    const int kn = min(kSmallKc, kend - k0);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) xs[8 * c + j][r] = f[j];
+    for (int q = 0; q < kSmallXLoads; ++q) {
+      const int i = tid + q * kSmallThreads;
+      const int r = i % kSmallTok, c = i / kSmallTok;  // consecutive threads: consecutive tokens
+      xr[q] = make_uint4(0u, 0u, 0u, 0u);
+      if (8 * c < kn && t0 + r < T) xr[q] = ld_v4(x + (size_t)(t0 + r) * H + k0 + 8 * c);
     }
-    const int w4 = kn / 4;
-    for (int i = tid; i < kSmallExp * w4; i += blockDim.x) {
+#pragma unroll
+    for (int q = 0; q < kSmallWLoads; ++q) {
+      const int i = tid + q * kSmallThreads;
       const int e = i % kSmallExp, c = i / kSmallExp;  // consecutive threads: consecutive experts
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e0 + e < E) v = __ldg(reinterpret_cast<const float4*>(wr + (size_t)(e0 + e) * H + k0) + c);
-      float* col = reinterpret_cast<float*>(&wsm[0][0]) + e;
-      col[(4 * c + 0) * kSmallExp] = v.x;
-      col[(4 * c + 1) * kSmallExp] = v.y;
-      col[(4 * c + 2) * kSmallExp] = v.z;
-      col[(4 * c + 3) * kSmallExp] = v.w;
+      wv[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (4 * c < kn && e0 + e < E)
+        wv[q] = __ldg(reinterpret_cast<const float4*>(wr + (size_t)(e0 + e) * H + k0) + c);
     }
-    __syncthreads();
+  };
+  // registers -> shared-memory buffer b
+  auto store = [&](int b) {
+    float* xs = xs_all + b * kSmallKc * kSmallTok;
+    float* ws = ws_all + b * kSmallKc * kSmallExp;
+#pragma unroll
+    for (int q = 0; q < kSmallXLoads; ++q) {
+      const int i = tid + q * kSmallThreads;
+      const int r = i % kSmallTok, c = i / kSmallTok;
+      float f[8];
+      unpack8(xr[q], f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xs[(8 * c + j) * kSmallTok + r] = f[j];
+    }
+#pragma unroll
+    for (int q = 0; q < kSmallWLoads; ++q) {
+      const int i = tid + q * kSmallThreads;
+      const int e = i % kSmallExp, c = i / kSmallExp;
+      ws[(4 * c + 0) * kSmallExp + e] = wv[q].x;
+      ws[(4 * c + 1) * kSmallExp + e] = wv[q].y;
+      ws[(4 * c + 2) * kSmallExp + e] = wv[q].z;
+      ws[(4 * c + 3) * kSmallExp + e] = wv[q].w;
+    }
+  };
+
+  load(kbeg);
+  store(0);
+  __syncthreads();
+  int b = 0;
+  for (int k0 = kbeg; k0 < kend; k0 += kSmallKc, b ^= 1) {
+    const bool more = k0 + kSmallKc < kend;
+    if (more) load(k0 + kSmallKc);
+    const int kn = min(kSmallKc, kend - k0);
+    const float* xs = xs_all + b * kSmallKc * kSmallTok;
+    const float4* ws = reinterpret_cast<const float4*>(ws_all + b * kSmallKc * kSmallExp);
     for (int kk = 0; kk < kn; ++kk) {
-      const float xv = xs[kk][tok];
-      const float4 w = wsm[kk][eg];
+      const float xv = xs[kk * kSmallTok + tok];
+      const float4 w = ws[kk * (kSmallExp / 4) + eg];
       acc[0] = fmaf(xv, w.x, acc[0]);
       acc[1] = fmaf(xv, w.y, acc[1]);
       acc[2] = fmaf(xv, w.z, acc[2]);
       acc[3] = fmaf(xv, w.w, acc[3]);
     }
+    // the other buffer was last read before the barrier that ended the previous chunk
+    if (more) store(b ^ 1);
     __syncthreads();
   }
   const int t = t0 + tok;
@@ -162,31 +209,64 @@ __device__ __forceinline__ void select_topk(const float (&v)[VPL], int E, int k,
   }
 }
 
-// One warp per token. Lane l holds logits of experts l, l+32, ...; VPL = values per lane.
+// Two warps per token (warp 2j: selection, warp 2j+1: shared gate and output row), so the
+// two latency chains run side by side. Lane l holds logits of experts l, l+32, ...;
+// VPL = values per lane, NS = partial-sum slices (a compile-time count, so that all
+// VPL * NS loads of a lane are in flight together).
 // `logits` holds `nslices` partial sums [nslices][T][E], added in slice order.
 // With `wr` set (logits from the tensor-core router, whose accumulation is not exact fp32),
 // a token whose k-th / (k+1)-th gap is below `band` has every expert whose logit lies within
 // `band` of the k-th recomputed as an exact fp32 dot product, and the selection is redone on
 // those values: the choice then matches fp32 arithmetic except at true near-ties.
-template <int VPL>
+template <int VPL, int NS>
 __global__ void __launch_bounds__(256)
-router_topk_kernel(const float* __restrict__ logits, int nslices, const float* __restrict__ bias,
+router_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
                    const uint16_t* __restrict__ x, const uint16_t* __restrict__ wsg,
                    const float* __restrict__ wr, float band, int T, int H, int E, int k,
                    int32_t* __restrict__ ids, float* __restrict__ w, float* __restrict__ sgate,
                    float* __restrict__ gap, float* __restrict__ out_zero) {
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int t = blockIdx.x * (blockDim.x >> 6) + (threadIdx.x >> 6);
   if (t >= T) return;
 
+  if ((threadIdx.x >> 5) & 1) {
+    // shared-expert gate: sigmoid(w_shared . x[t])
+    float g = 0.f;
+    const uint16_t* xr = x + (size_t)t * H;
+#pragma unroll 4
+    for (int c = lane; c < H / 8; c += 32) {
+      const uint4 xa = ld_v4(xr + 8 * c);
+      const uint4 wa = ld_v4(wsg + 8 * c);
+      float xf[8];
+      unpack8(xa, xf);
+      g = dot8_acc(wa, xf, g);
+    }
+    g = warp_sum(g);
+    if (lane == 0) sgate[t] = 1.f / (1.f + expf(-g));
+    if (out_zero) {
+      float4* o = reinterpret_cast<float4*>(out_zero + (size_t)t * H);
+      for (int c = lane; c < H / 4; c += 32) o[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
+
+  float part[NS][VPL];
+#pragma unroll
+  for (int sl = 0; sl < NS; ++sl)
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane + 32 * i;
+      part[sl][i] = e < E ? logits[((size_t)sl * T + t) * E + e] : 0.f;
+    }
   float v[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
     float l = -FLT_MAX;
     if (e < E) {
-      l = logits[(size_t)t * E + e];
-      for (int sl = 1; sl < nslices; ++sl) l += logits[((size_t)sl * T + t) * E + e];
+      l = part[0][i];
+#pragma unroll
+      for (int sl = 1; sl < NS; ++sl) l += part[sl][i];
       if (bias) l += bias[e];
     }
     v[i] = l;
@@ -226,24 +306,6 @@ router_topk_kernel(const float* __restrict__ logits, int nslices, const float* _
   }
   const float kth = __shfl_sync(0xffffffffu, my_val, k - 1);
   if (gap && lane == 0) gap[t] = (k < E) ? kth - next_val : __int_as_float(0x7f800000);
-
-  // shared-expert gate: sigmoid(w_shared . x[t])
-  float g = 0.f;
-  const uint16_t* xr = x + (size_t)t * H;
-  for (int c = lane; c < H / 8; c += 32) {
-    const uint4 xa = ld_v4(xr + 8 * c);
-    const uint4 wa = ld_v4(wsg + 8 * c);
-    float xf[8];
-    unpack8(xa, xf);
-    g = dot8_acc(wa, xf, g);
-  }
-  g = warp_sum(g);
-  if (lane == 0) sgate[t] = 1.f / (1.f + expf(-g));
-
-  if (out_zero) {
-    float4* o = reinterpret_cast<float4*>(out_zero + (size_t)t * H);
-    for (int c = lane; c < H / 4; c += 32) o[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
 }
 
 }  // namespace
@@ -263,9 +325,17 @@ cudaError_t launch_router_logits(const moe_shape& s, const Layout& L, char* ws, 
   const int nslices = router_slices(s);
   const bool tc_logits = nslices == 1 && tc_router_supported(s);
   if (nslices == 1 && tc_router_supported(s)) return launch_tc_router(s, L, ws, x, wr, logits, st);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(router_logits_small_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmem);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
   LaunchScope scope(MOE_K_ROUTER_LOGITS, st);
   dim3 grid((s.E + kSmallExp - 1) / kSmallExp, nslices, (s.T + kSmallTok - 1) / kSmallTok);
-  router_logits_small_kernel<<<grid, 256, 0, st>>>(x, wr, logits, s.T, s.H, s.E, nslices);
+  router_logits_small_kernel<<<grid, kSmallThreads, kSmallSmem, st>>>(x, wr, logits, s.T, s.H,
+                                                                      s.E, nslices);
   return cudaGetLastError();
 }
 
@@ -276,13 +346,22 @@ cudaError_t launch_router_topk(const moe_shape& s, const float* logits, const fl
   LaunchScope scope(MOE_K_ROUTER_TOPK, st);
   const int nslices = router_slices(s);
   const bool tc_logits = nslices == 1 && tc_router_supported(s);
-  const int warps = 8;
-  dim3 grid((s.T + warps - 1) / warps);
+  // two warps per token; one token per CTA for small batches so that they spread over SMs
+  const int tpb = s.T < kTcRouterMinTokens ? 1 : 4;
+  const int warps = 2 * tpb;
+  dim3 grid((s.T + tpb - 1) / tpb);
   const int vpl = (s.E + 31) / 32;
 #define MOE_TOPK_CASE(N)                                                                     \
-  router_topk_kernel<N><<<grid, warps * 32, 0, st>>>(logits, nslices, bias, x, wsg,             \
-                                                     tc_logits ? wr : nullptr, kRefineBand, s.T, s.H, \
-                                                     s.E, s.k, ids, w, sgate, gap, out_zero)
+  do {                                                                                       \
+    if (nslices == kSplits)                                                                  \
+      router_topk_kernel<N, kSplits><<<grid, warps * 32, 0, st>>>(                             \
+          logits, bias, x, wsg, nullptr, kRefineBand, s.T, s.H, s.E, s.k, ids, w, sgate, gap,  \
+          out_zero);                                                                         \
+    else                                                                                     \
+      router_topk_kernel<N, 1><<<grid, warps * 32, 0, st>>>(                                   \
+          logits, bias, x, wsg, tc_logits ? wr : nullptr, kRefineBand, s.T, s.H, s.E, s.k, ids, \
+          w, sgate, gap, out_zero);                                                          \
+  } while (0)
   if (vpl <= 1) MOE_TOPK_CASE(1);
   else if (vpl <= 2) MOE_TOPK_CASE(2);
   else if (vpl <= 4) MOE_TOPK_CASE(4);
