@@ -50,7 +50,7 @@ KERNEL_SOURCES = {  # kernel id -> source file whose hash a stored ncu traffic f
 }
 # oracle token sample per workload for the CPU baseline (about 10-30 s on a host)
 CPU_SAMPLE = {"tiny": 64, "flash_decode": 16, "flash_prefill": 32, "flash_prefill_e64": 32,
-              "t24_prefill": 3, "t24_skewed": 3}
+              "t24_prefill_e16": 3, "t24_prefill": 3, "t24_skewed": 3}
 
 
 def log(*a):
