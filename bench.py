@@ -41,9 +41,9 @@ METRIC = "MoE-layer tokens/s (prefill), µs/layer (decode); % of TC or HBM roofl
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {  # kernel id -> source file whose hash a stored ncu traffic figure carries
-    "gate_up": ("stream_swiglu.cu", "tc_gemm.cu"),
-    "down": ("stream_swiglu.cu", "tc_gemm.cu"),
-    "router_logits": ("router.cu", "tc_gemm.cu"),
+    "gate_up": ("stream_swiglu.cu", "tc_gemm.cu", "tc2_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
+    "down": ("stream_swiglu.cu", "tc_gemm.cu", "tc2_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
+    "router_logits": ("router.cu", "tc_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
     "router_topk": ("router.cu",),
     "permute": ("permute.cu",),
     "combine": ("combine.cu",),
@@ -287,7 +287,7 @@ def run_ours(args, cfg, world, rank, local):
     import synth
 
     variant = {"auto": moe.MOE_VARIANT_AUTO, "stream": moe.MOE_VARIANT_STREAM,
-               "tc": moe.MOE_VARIANT_TC}[args.variant]
+               "tc": moe.MOE_VARIANT_TC, "tc2": moe.MOE_VARIANT_TC2}[args.variant]
     moe.moe_set_variant(variant)
     dev = synth.device_inputs(cfg, seed=0, x_seed=rank, device=f"cuda:{local}")
     s = moe.shape_of(cfg)
@@ -449,7 +449,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="flash_decode", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--variant", default="auto", choices=["auto", "stream", "tc"])
+    ap.add_argument("--variant", default="auto", choices=["auto", "stream", "tc", "tc2"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel from the host")
     args = ap.parse_args()

@@ -33,6 +33,7 @@ MOE_ERR_DEVICE_BOUNDS = 6
 MOE_VARIANT_AUTO = 0
 MOE_VARIANT_STREAM = 1
 MOE_VARIANT_TC = 2
+MOE_VARIANT_TC2 = 3
 
 KERNELS = ("router_logits", "router_topk", "permute", "gate_up", "down", "combine", "other")
 MOE_K_COUNT = len(KERNELS)

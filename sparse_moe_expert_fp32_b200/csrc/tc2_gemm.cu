@@ -1,0 +1,517 @@
+// tc2_gemm.cu -- stage 4, "Grouped expert GEMMs" (Qwen3.8-Flash-Next architecture study,
+// MoE pipeline diagram; expert(x) = W_down(SiLU(W_gate x) * W_up x)) for prefill-size
+// batches, on CTA pairs: one tcgen05.mma.cta_group::2 (M = 256) per 16-wide K step spans
+// two SMs, each holding 128 rows of the weight tile and HALF of the token tile in its own
+// shared memory.
+//
+// Why pairs: with ~160 tokens per expert the one-SM kernels are bound by shared-memory
+// bandwidth (TMA writes plus the operand reads of every MMA at 128 bytes per clock), not by
+// the tensor cores. A pair halves each SM's share of the token operand, and the down GEMM
+// folds the hi and lo halves of h into the N dimension of one MMA, so its weight tile is
+// read from shared memory once instead of twice.
+//
+//   gate|up (pair tile: 128 channels x up to 256 tokens of one expert). CTA r holds gate rows
+//     [c + 64r, c + 64r + 64) and the up rows of the same channels as its 128 A rows, and
+//     token rows [N/2 r, N/2 (r + 1)) of the tile as its B half. Tensor-memory lanes 0-63
+//     then hold gate and lanes 64-127 up for the same 64 channels; the epilogue pairs a
+//     gate warp with an up warp through shared memory and stores h = SiLU(gate) * up as
+//     the bf16 pair hi = bf16(h), lo = bf16(h - hi).
+//   down (pair tile: 256 output channels x up to 128 packed rows). CTA r holds W_down rows
+//     [m + 128r, m + 128r + 128) and plane r of h (r = 0: hi, r = 1: lo) for the tile's
+//     rows, so the MMA's N = 2 x rows: columns [0, N) are W h_hi, [N, 2N) are W h_lo, and
+//     the epilogue adds the two before scaling by the routing weight and adding into out.
+//
+// Roles in each 320-thread CTA (one CTA per SM, persistent; pair p takes tiles p, p + P,
+// p + 2P, ... of the plan's order, so neighbouring tiles run at the same time):
+//   warp 0      TMA producer over a ring of 6 stages (32 KB: 128 A rows + up to 128 B rows
+//               of 64 K each); both CTAs count their copies on the leader's full barrier;
+//   warp 1      tensor memory (512 columns, two 256-column slots, allocated for the pair);
+//               in the leader CTA lane 0 issues the pair MMAs and commits them to both CTAs;
+//   warps 2..9  epilogue; warp w reads TMEM lanes 32*(w%4) .. +31; the first four warps
+//               take even 32-column chunks, the last four odd ones.
+// Every mbarrier wait is bounded (2 s); on expiry the kernel records the timeout flag and
+// every role leaves; the pair meets at a final cluster barrier before freeing TMEM.
+#include <algorithm>
+
+#include "tc_common.cuh"
+#include "tc_gemm.h"
+
+namespace moe {
+namespace {
+
+constexpr int kEpi = 8;
+constexpr int kThreads2 = 64 + 32 * kEpi;
+constexpr int kBK = 64;                       // K per stage: 128-byte rows, 128-byte swizzle
+constexpr uint32_t kRowB = kBK * 2;
+constexpr uint32_t kABytes = 128u * kRowB;    // this CTA's 128 weight rows
+constexpr uint32_t kBBytes = 128u * kRowB;    // this CTA's token half, at most 128 rows
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr int kStages = 6;
+constexpr int kSlotCols = 256;
+constexpr int kBoxes = 5;  // token boxes of 128, 64, 32, 16 and 8 rows
+__host__ __device__ constexpr int box_rows(int i) { return 128 >> i; }
+
+enum PairMode { kPairGateUp = 0, kPairDown = 1 };
+
+struct PairShared {
+  uint64_t full[kStages];   // leader: both CTAs' copies of a stage have landed
+  uint64_t empty[kStages];  // each CTA: the MMAs reading its copy of a stage are done
+  uint64_t tmem_full[2];    // each CTA: the accumulator slot holds a finished tile
+  uint64_t tmem_empty[2];   // leader: both CTAs' epilogues have drained the slot
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort;
+  int tp[kMaxE + 2];
+  int row0[kMaxE + 2];
+  union {
+    float4 xpose[kEpi][8][8];  // down: per warp, 8 tokens x 32 channels
+    float up[4][32][32];       // gate|up: per warp pair, 32 tokens x 32 channels of up
+  };
+};
+
+constexpr size_t pair_smem_bytes() {
+  return 1024 + (size_t)kStages * kStageBytes + sizeof(PairShared);
+}
+static_assert(pair_smem_bytes() <= 232448, "over the 227 KB of shared memory a CTA may use");
+
+struct PairMaps {
+  CUtensorMap m[kBoxes];
+};
+
+// This CTA's token half of an nb-row B operand as boxes of 128/64/32/16/8 rows: piece j's
+// first row and box index; false past the last piece (nb is a multiple of 8, at most 128).
+__device__ __forceinline__ bool b_piece(int nb, int j, int& row, int& bidx) {
+  int r = 0;
+#pragma unroll
+  for (int i = 0; i < kBoxes; ++i) {
+    if (nb & box_rows(i)) {
+      if (j == 0) {
+        row = r;
+        bidx = i;
+        return true;
+      }
+      --j;
+      r += box_rows(i);
+    }
+  }
+  return false;
+}
+
+struct PairGeom {
+  Tile t;
+  int a_row0, a_row1;  // gate|up: the 64 gate and 64 up rows; down: 128 rows from a_row0
+  int b_row;           // first row of this CTA's token half in its tensor map
+  int nb;              // rows of this CTA's token half
+  int n_mma;           // MMA N
+  int nk;              // K stages
+  bool shared;
+};
+
+template <int MODE>
+__device__ __forceinline__ PairGeom pair_geom(const TcArgs& a, const PairShared& S, int tile,
+                                              int R, int rank, int plane_rows) {
+  PairGeom G;
+  G.t = decode_tile(S.row0, S.tp, a.E, tile, MODE == kPairGateUp ? 256 : 128);
+  G.shared = G.t.g == a.E;
+  if (MODE == kPairGateUp) {
+    const int Ig = G.shared ? a.Is : a.I;
+    const int base = G.shared ? 0 : G.t.g * 2 * a.I;
+    G.a_row0 = base + G.t.m * 128 + rank * 64;
+    G.a_row1 = G.a_row0 + Ig;
+    G.nb = G.t.N / 2;
+    G.b_row = (G.shared ? G.t.p0 - R : G.t.p0) + rank * G.nb;
+    G.n_mma = G.t.N;
+    G.nk = a.H / kBK;
+  } else {
+    const int base = G.shared ? 0 : G.t.g * a.H;
+    G.a_row0 = base + G.t.m * 256 + rank * 128;
+    G.a_row1 = 0;
+    G.nb = G.t.N;
+    G.b_row = G.t.p0 + rank * plane_rows;
+    G.n_mma = 2 * G.t.N;
+    G.nk = (G.shared ? a.Is : a.I) / kBK;
+  }
+  return G;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads2, 1)
+tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_sh,
+                   const __grid_constant__ PairMaps tm_b, const __grid_constant__ PairMaps tm_b_sh,
+                   const TcArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  PairShared& S = *reinterpret_cast<PairShared*>(smem + kStages * kStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = (int)ptx::cluster_ctarank();  // 0: the leader, which issues the MMAs
+  const int pair = (int)ptx::cluster_id_x(), npairs = (int)ptx::cluster_count_x();
+  const int E = args.E;
+  const PlanView pv = plan_view(const_cast<int*>(args.plan), E);
+  const int* tp = (MODE == kPairGateUp) ? pv.tp1 : pv.tp2;
+  for (int g = threadIdx.x; g < E + 2; g += blockDim.x) {
+    S.tp[g] = tp[g];
+    S.row0[g] = pv.row0[g];
+  }
+  const int total = tp[E + 1];
+  const int R = pv.row0[E];
+  const int plane_rows = (MODE == kPairDown) ? (int)(args.h_plane / (size_t)args.ldh) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(&S.full[s], 1);
+      ptx::mbar_init(&S.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&S.tmem_full[b], 1);
+      ptx::mbar_init(&S.tmem_empty[b], 2 * kEpi);  // one lane per epilogue warp of both CTAs
+    }
+    ptx::mbar_init(&S.drain, 1);
+    S.abort = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tm_a);
+    ptx::prefetch_tmap(&tm_a_sh);
+    for (int i = 0; i < kBoxes; ++i) {
+      ptx::prefetch_tmap(&tm_b.m[i]);
+      ptx::prefetch_tmap(&tm_b_sh.m[i]);
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(&S.tmem_base, 512);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // the peer's barriers exist before anyone signals them
+  ptx::tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    // Lane 0 waits for this CTA's copy of a stage to be free (and in the leader arms the
+    // full barrier with both CTAs' bytes); then each lane with a box issues it: lanes 0-1
+    // the weight rows, lanes 2.. the pieces of this CTA's token half.
+    const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(&S.full[0]), 0);
+    int it = 0;
+    bool aborted = false;
+    for (int tile = pair; tile < total && !aborted; tile += npairs) {
+      const PairGeom G = pair_geom<MODE>(args, S, tile, R, rank, plane_rows);
+      const CUtensorMap* my_map = nullptr;
+      uint32_t my_off = 0;
+      int my_row = 0;
+      if (MODE == kPairGateUp && lane < 2) {  // 64 gate rows, then 64 up rows
+        my_map = G.shared ? &tm_a_sh : &tm_a;
+        my_off = lane * (kABytes / 2);
+        my_row = lane ? G.a_row1 : G.a_row0;
+      } else if (MODE == kPairDown && lane == 0) {
+        my_map = G.shared ? &tm_a_sh : &tm_a;
+        my_row = G.a_row0;
+      } else if (lane >= 2) {
+        int r, bi;
+        if (b_piece(G.nb, lane - 2, r, bi)) {
+          const PairMaps& bm = (MODE == kPairGateUp && G.shared) ? tm_b_sh : tm_b;
+          my_map = &bm.m[bi];
+          my_off = kABytes + (uint32_t)r * kRowB;
+          my_row = G.b_row + r;
+        }
+      }
+      const uint32_t bytes = 2u * (kABytes + (uint32_t)G.nb * kRowB);  // both CTAs
+      for (int ks = 0; ks < G.nk; ++ks, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        bool ok = true;
+        if (lane == 0) {
+          ok = wait_phase(&S.empty[s], ph ^ 1u, S, args.status);
+          if (ok && rank == 0) ptx::mbar_arrive_expect_tx(&S.full[s], bytes);
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          aborted = true;
+          break;
+        }
+        if (my_map)
+          ptx::tma_load_2d_pair(smem + s * kStageBytes + my_off, my_map,
+                                full0 + (uint32_t)(s * sizeof(uint64_t)), ks * kBK, my_row);
+      }
+    }
+    // wait until the MMAs have released every stage this CTA filled, so that no commit
+    // from the leader is still on its way to this CTA's barriers when the pair leaves
+    if (lane == 0 && !aborted) {
+      for (int j = 0; j < kStages && j < it; ++j) {
+        const int u = it - 1 - j;
+        if (!wait_phase(&S.empty[u % kStages], (uint32_t)(u / kStages) & 1u, S, args.status))
+          break;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ pair MMA issuer (leader)
+    if (rank == 0 && lane == 0) {
+      int it = 0, nt = 0;
+      bool aborted = false;
+      for (int tile = pair; tile < total && !aborted; tile += npairs, ++nt) {
+        const PairGeom G = pair_geom<MODE>(args, S, tile, R, rank, plane_rows);
+        const int slot = nt & 1;
+        const uint32_t use = (uint32_t)(nt >> 1);
+        if (!wait_phase(&S.tmem_empty[slot], (use & 1u) ^ 1u, S, args.status)) {
+          aborted = true;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(slot * kSlotCols);
+        const uint32_t idesc = ptx::idesc_bf16_f32(256, G.n_mma);
+        for (int ks = 0; ks < G.nk; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          // The copies' completion on the full barrier orders them before the MMAs that read
+          // the stage; no tcgen05 fence is needed here (one per stage serialised the MMAs).
+          // A non-blocking test first: a stage that has landed costs no suspended wait.
+          if (!ptx::mbar_test_wait(&S.full[s], ph) && !wait_phase(&S.full[s], ph, S, args.status)) {
+            aborted = true;
+            break;
+          }
+          const uint8_t* st = smem + s * kStageBytes;
+          const uint64_t ad = ptx::smem_desc_kmajor<kRowB>(st);
+          const uint64_t bd = ptx::smem_desc_kmajor<kRowB>(st + kABytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes along K = +2 in the address field
+            ptx::umma_bf16_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          ptx::umma_commit_pair(&S.empty[s], 0x3);
+        }
+        if (aborted) break;
+        ptx::umma_commit_pair(&S.tmem_full[slot], 0x3);
+      }
+      if (aborted) {
+        ptx::umma_commit_pair(&S.drain, 0x1);  // completes once every MMA issued so far is done
+        drain_phase(&S.drain, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;  // which 32-column chunks this warp drains
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t tmem_empty0 = ptx::mapa_shared(ptx::smem_u32(&S.tmem_empty[0]), 0);
+    // gate|up: warps q = 0, 1 hold gate and q = 2, 3 up of the same 32 channels
+    const int xp = half * 2 + (q & 1);  // warp pair index, 0..3
+    // named barriers of the pair: its per-tile decision, "buffer free", "buffer full"
+    const int bar_dec = 1 + 3 * xp, bar_free = 2 + 3 * xp, bar_full = 3 + 3 * xp;
+    int nt = 0;
+    for (int tile = pair; tile < total; tile += npairs, ++nt) {
+      const PairGeom G = pair_geom<MODE>(args, S, tile, R, rank, plane_rows);
+      const Tile& tl = G.t;
+      const int slot = nt & 1;
+      const uint32_t use = (uint32_t)(nt >> 1);
+      const uint32_t base = tmem + lane_off + (uint32_t)(slot * kSlotCols);
+      // down: token and weight of this warp's columns, requested before waiting for the
+      // accumulator so that the loads overlap the tile's MMAs
+      int col_tok[2] = {0, 0};
+      float col_w[2] = {0.f, 0.f};
+      if (MODE == kPairDown) {
+#pragma unroll
+        for (int ci = 0; ci < 2; ++ci) {
+          const int c = (2 * ci + half) * 32 + lane;
+          if (c < tl.nvalid) {
+            const int p = tl.p0 + c;
+            col_tok[ci] = token_of_row(args, p, R);
+            if (args.out) col_w[ci] = p < R ? args.sorted_w[p] : args.sgate[col_tok[ci]];
+          }
+        }
+      }
+      bool ok = wait_phase(&S.tmem_full[slot], use & 1u, S, args.status);
+      // the gate and up warps of a pair decide together (they meet at named barriers below)
+      ok = (MODE == kPairGateUp) ? ptx::bar_and(bar_dec, 64, ok) : __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (MODE == kPairGateUp) {
+        const int ch = tl.m * 128 + rank * 64 + (q & 1) * 32 + lane;  // this lane's channel
+        float(&xu)[32][32] = S.up[xp];
+#pragma unroll 1
+        for (int ci = 0; ci < 4; ++ci) {
+          const int c0 = (2 * ci + half) * 32;
+          if (c0 >= tl.nvalid) break;
+          uint32_t r[32];
+          ptx::tmem_ld32(base + (uint32_t)c0, r);
+          ptx::tmem_ld_wait();
+          if (q >= 2) {  // up warp: hand its 32 x 32 values to the gate warp
+            ptx::bar_sync(bar_free, 64);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) xu[j][lane] = __uint_as_float(r[j]);
+            ptx::bar_arrive(bar_full, 64);
+          } else {
+            ptx::bar_arrive(bar_free, 64);
+            ptx::bar_sync(bar_full, 64);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (c0 + j < tl.nvalid) {
+                const float gv = __uint_as_float(r[j]);
+                // SiLU(g) = g / (1 + e^-g) with the fast exponential and division (a few
+                // ulp; h is carried with about 16 significant bits)
+                const float hv = __fdividef(gv, 1.f + __expf(-gv)) * xu[j][lane];
+                const uint16_t hi = f32_to_bf16_rn(hv);
+                const size_t at = (size_t)(tl.p0 + c0 + j) * args.ldh + ch;
+                args.h[at] = hi;
+                args.h[args.h_plane + at] = f32_to_bf16_rn(hv - bf16lo(hi));
+              }
+            }
+          }
+        }
+      } else {
+        // columns [0, N) hold W h_hi and [N, 2N) W h_lo of the same rows
+        const int mrow = tl.m * 256 + rank * 128 + q * 32 + 4 * (lane & 7);  // this lane's channels
+        const int H = args.H;
+        float4(&xpz)[8][8] = S.xpose[warp - 2];
+#pragma unroll
+        for (int ci = 0; ci < 2; ++ci) {
+          const int c0 = (2 * ci + half) * 32;
+          if (c0 >= tl.nvalid) break;
+          uint32_t r0[32], r1[32];
+          ptx::tmem_ld32(base + (uint32_t)c0, r0);
+          ptx::tmem_ld32(base + (uint32_t)(tl.N + c0), r1);
+          ptx::tmem_ld_wait();
+          // 32 channels (lanes) x 32 tokens (registers); every 8 tokens go through shared
+          // memory so that eight lanes own the 32 channels (128 bytes) of one token and each
+          // 16-byte atomic add of a warp lands in whole 128-byte lines
+#pragma unroll
+          for (int sb = 0; sb < 4; ++sb) {
+            __syncwarp();
+            float* xs = reinterpret_cast<float*>(&xpz[0][0]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              xs[k * 32 + lane] = __uint_as_float(r0[sb * 8 + k]) + __uint_as_float(r1[sb * 8 + k]);
+            __syncwarp();
+#pragma unroll
+            for (int hq = 0; hq < 2; ++hq) {
+              const int k = hq * 4 + (lane >> 3);  // this lane's token within the 8
+              const float4 v = xpz[k][lane & 7];
+              const int col = c0 + sb * 8 + k;
+              const int t = __shfl_sync(0xffffffffu, col_tok[ci], sb * 8 + k);
+              const float w = __shfl_sync(0xffffffffu, col_w[ci], sb * 8 + k);
+              if (col < tl.nvalid) {
+                const int p = tl.p0 + col;
+                if (args.out) {
+                  atomicAdd(reinterpret_cast<float4*>(args.out + (size_t)t * H + mrow),
+                            make_float4(w * v.x, w * v.y, w * v.z, w * v.w));
+                } else {
+                  float* row =
+                      p < R ? args.y + (size_t)p * H : args.y_shared + (size_t)(p - R) * H;
+                  *reinterpret_cast<float4*>(row + mrow) = v;
+                }
+              }
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(tmem_empty0 + (uint32_t)(slot * sizeof(uint64_t)));
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (S.abort) {
+    // copies or commits aimed at the pair's barriers may still be in flight: give them time
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) {
+    }
+  }
+  ptx::cluster_sync();  // neither CTA frees TMEM or leaves while its peer may signal it
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+bool make_pair_maps(PairMaps* b, const void* base, uint64_t inner, uint64_t outer) {
+  for (int i = 0; i < kBoxes; ++i)
+    if (!make_map(&b->m[i], base, inner, outer, kBK, (uint32_t)box_rows(i))) return false;
+  return true;
+}
+
+template <int MODE>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& a_sh, const PairMaps& b,
+                        const PairMaps& b_sh, const TcArgs& args, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int max_pairs = 0;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(tc2_grouped_kernel<MODE>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)pair_smem_bytes());
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (unsigned)sm_count(), 1, 1);
+    cfg.blockDim = dim3(kThreads2, 1, 1);
+    cfg.dynamicSmemBytes = pair_smem_bytes();
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    attr_err = cudaOccupancyMaxActiveClusters(&max_pairs, tc2_grouped_kernel<MODE>, &cfg);
+    if (attr_err == cudaSuccess && max_pairs < 1) attr_err = cudaErrorInvalidConfiguration;
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * (unsigned)max_pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads2, 1, 1);
+  cfg.dynamicSmemBytes = pair_smem_bytes();
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc2_grouped_kernel<MODE>, a, a_sh, b, b_sh, args);
+}
+
+}  // namespace
+
+cudaError_t launch_tc2_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
+                               const int32_t* sorted_token, const moe_weights& w,
+                               cudaStream_t st) {
+  uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
+  cudaError_t e = launch_gather_rows(s, L, ws, x, sorted_token, st);
+  if (e != cudaSuccess) return e;
+  CUtensorMap a, a_sh;
+  PairMaps b, b_sh;
+  if (!make_map(&a, w.w_gate_up, s.H, (uint64_t)s.E * 2 * s.I, kBK, 64) ||
+      !make_map(&a_sh, w.ws_gate_up, s.H, 2ull * s.Is, kBK, 64) ||
+      !make_pair_maps(&b, xs, s.H, (uint64_t)s.T * s.k) ||
+      !make_pair_maps(&b_sh, x, s.H, (uint64_t)s.T))
+    return cudaErrorInvalidValue;
+  TcArgs args = base_args(s, L, ws);
+  args.sorted_token = sorted_token;
+  LaunchScope scope(MOE_K_GATE_UP, st);
+  return launch_pair<kPairGateUp>(a, a_sh, b, b_sh, args, st);
+}
+
+cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
+                            const int32_t* sorted_token, const float* sorted_w, const float* sgate,
+                            const moe_weights& w, float* y, float* y_shared, float* out,
+                            cudaStream_t st) {
+  CUtensorMap a, a_sh;
+  PairMaps b;
+  if (!make_map(&a, w.w_down, s.I, (uint64_t)s.E * s.H, kBK, 128) ||
+      !make_map(&a_sh, w.ws_down, s.Is, (uint64_t)s.H, kBK, 128) ||
+      !make_pair_maps(&b, ws + L.h, L.ldh, 2 * (L.h_plane / L.ldh)))
+    return cudaErrorInvalidValue;
+  TcArgs args = base_args(s, L, ws);
+  args.sorted_token = sorted_token;
+  args.sorted_w = sorted_w;
+  args.sgate = sgate;
+  args.y = y;
+  args.y_shared = y_shared;
+  args.out = out;
+  LaunchScope scope(MOE_K_DOWN, st);
+  return launch_pair<kPairDown>(a, a_sh, b, b, args, st);
+}
+
+}  // namespace moe

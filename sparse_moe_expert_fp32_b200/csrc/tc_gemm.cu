@@ -32,14 +32,9 @@
 //               even 32-column chunks, the last four odd ones.
 // Every mbarrier wait is bounded (2 s); on expiry the kernel records the timeout flag,
 // lets every role leave its loop, drains its own copies and MMAs and frees TMEM.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <algorithm>
-#include <mutex>
 
-#include "device_common.cuh"
-#include "sm100_ptx.cuh"
+#include "tc_common.cuh"
 #include "tc_gemm.h"
 
 namespace moe {
@@ -53,8 +48,6 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 // the token loads the slowest part of a prefill stage.
 constexpr int kBoxHeights = 4;
 __host__ __device__ constexpr int box_rows_of(int i) { return 128 >> i; }
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr uint64_t kDrainLimitNs = 200000000ull;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256;
 constexpr int kQueue = 4;  // tile ids handed from the producer to the MMA and epilogue roles
@@ -130,91 +123,6 @@ __device__ __forceinline__ bool token_piece(int N, int j, int& row, int& hidx) {
     }
   }
   return false;
-}
-
-struct TcArgs {
-  const int* plan;
-  int E, H, I, Is, T, ldh;
-  size_t h_plane;
-  const int32_t* sorted_token;
-  const float* sorted_w;
-  const float* sgate;
-  uint16_t* h;
-  float* y;
-  float* y_shared;
-  float* out;
-  uint32_t* status;
-  float* logits;      // router: [T][E]
-  int ntiles;         // router: tile count (no plan)
-  int* counter;       // next tile to hand out (zeroed before the launch)
-  int* counter_next;  // gate|up: the down kernel's counter, zeroed here for its launch
-};
-
-struct Tile {
-  int g, m, p0, nvalid, N;
-};
-
-// Tile -> (group, M tile, packed rows). Groups own consecutive tile ranges
-// [tp[g], tp[g+1]); a group of more than max_tile rows is split into near-equal chunks
-// whose tiles are adjacent.
-__device__ __forceinline__ Tile decode_tile(const int* row0, const int* tp, int E, int tile,
-                                            int max_tile) {
-  int lo = 0, hi = E + 1;  // tp[lo] <= tile < tp[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (tp[mid] <= tile) lo = mid;
-    else hi = mid;
-  }
-  Tile t;
-  t.g = lo;
-  const int n = row0[lo + 1] - row0[lo];
-  const int nch = (n + max_tile - 1) / max_tile;
-  const int cs = (((n + nch - 1) / nch) + 15) & ~15;
-  const int local = tile - tp[lo];
-  t.m = local / nch;
-  const int c = local - t.m * nch;
-  const int start = c * cs;
-  t.nvalid = min(cs, n - start);
-  t.N = (t.nvalid + 15) & ~15;
-  t.p0 = row0[lo] + start;
-  return t;
-}
-
-// Bounded wait on an mbarrier phase; false if it ran out (flag recorded) or another role
-// already gave up.
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, SharedState& S,
-                                           uint32_t* status) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t spin = 1;; ++spin) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((spin & 31) == 0) {
-      if (S.abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        S.abort = 1;
-        set_flag(status, kFlagTimeout);
-        return false;
-      }
-    }
-  }
-}
-
-// Short bounded wait used while leaving after an abort.
-__device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!ptx::mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
-  }
-}
-
-__device__ __forceinline__ int token_of_row(const TcArgs& a, int p, int R) {
-  if (p >= R) return p - R;
-  const int t = a.sorted_token[p];
-  if ((unsigned)t >= (unsigned)a.T) {
-    set_flag(a.status, kFlagBounds);
-    return 0;
-  }
-  return t;
 }
 
 // Everything the three roles need to know about one tile.
@@ -451,11 +359,13 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         for (int ks = 0; ks < G.nk; ++ks, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
-          if (!wait_phase(&S.full[s], ph, S, args.status)) {
+          // The copies' completion on the full barrier orders them before the MMAs that read
+          // the stage; no tcgen05 fence is needed here (one per stage serialised the MMAs).
+          // A non-blocking test first: a stage that has landed costs no suspended wait.
+          if (!ptx::mbar_test_wait(&S.full[s], ph) && !wait_phase(&S.full[s], ph, S, args.status)) {
             aborted = true;
             break;
           }
-          ptx::tc_fence_after();
           const uint8_t* st = smem + s * C::kStageBytes;
           const uint64_t a0 = ptx::smem_desc_kmajor<C::kRowBytes>(st);
           const uint64_t a1 = ptx::smem_desc_kmajor<C::kRowBytes>(st + C::kATileBytes);
@@ -665,49 +575,11 @@ __global__ void router_split_kernel(const float* __restrict__ wr, uint16_t* __re
 
 // ---------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 2-D bf16 tensor [outer][inner] (inner contiguous), box [box_outer][box_inner] with the
-// swizzle matching box_inner (64 elements: 128-byte swizzle, 32: 64-byte swizzle).
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-              uint32_t box_inner, uint32_t box_outer) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * sizeof(uint16_t)};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapSwizzle sw =
-      box_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // The token tensor [outer][inner] in every box height of a token tile.
 bool make_bmaps(BMaps* b, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner) {
   for (int i = 0; i < kBoxHeights; ++i)
     if (!make_map(&b->m[i], base, inner, outer, box_inner, (uint32_t)box_rows_of(i))) return false;
   return true;
-}
-
-int sm_count() {
-  int dev = 0, n = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n;
 }
 
 template <int MODE>
@@ -723,21 +595,6 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& a_sh, const BMa
   if (attr_err != cudaSuccess) return attr_err;
   tc_grouped_kernel<MODE><<<grid, kThreads, smem_bytes<MODE>(), st>>>(a, a_sh, b, b_sh, args);
   return cudaGetLastError();
-}
-
-TcArgs base_args(const moe_shape& s, const Layout& L, char* ws) {
-  TcArgs a{};
-  a.plan = reinterpret_cast<const int*>(ws + L.plan);
-  a.E = s.E;
-  a.H = s.H;
-  a.I = s.I;
-  a.Is = s.Is;
-  a.T = s.T;
-  a.ldh = L.ldh;
-  a.h_plane = L.h_plane;
-  a.h = reinterpret_cast<uint16_t*>(ws + L.h);
-  a.status = reinterpret_cast<uint32_t*>(ws + L.status);
-  return a;
 }
 
 }  // namespace
@@ -781,16 +638,22 @@ bool tc_supported(const moe_shape& s) {
   return tc_router_supported(s);
 }
 
+cudaError_t launch_gather_rows(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
+                               const int32_t* sorted_token, cudaStream_t st) {
+  LaunchScope scope(MOE_K_OTHER, st);
+  gather_rows_kernel<<<sm_count() * 8, 256, 0, st>>>(
+      x, sorted_token, reinterpret_cast<const int*>(ws + L.plan), s.E, s.T, s.H,
+      reinterpret_cast<uint16_t*>(ws + L.xs), reinterpret_cast<uint32_t*>(ws + L.status),
+      reinterpret_cast<int*>(ws + L.sched) + 0);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                               const int32_t* sorted_token, const moe_weights& w, cudaStream_t st) {
   using C = Cfg<kGateUp>;
   uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
   {
-    LaunchScope scope(MOE_K_OTHER, st);
-    gather_rows_kernel<<<sm_count() * 8, 256, 0, st>>>(
-        x, sorted_token, reinterpret_cast<const int*>(ws + L.plan), s.E, s.T, s.H, xs,
-        reinterpret_cast<uint32_t*>(ws + L.status), reinterpret_cast<int*>(ws + L.sched) + 0);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_gather_rows(s, L, ws, x, sorted_token, st);
     if (e != cudaSuccess) return e;
   }
   CUtensorMap a, a_sh;

@@ -20,4 +20,18 @@ cudaError_t launch_tc_down(const moe_shape& s, const Layout& L, char* ws,
                            const moe_weights& w, float* y, float* y_shared, float* out,
                            cudaStream_t st);
 
+// Token rows in dispatch order (xs[p] = x[sorted_token[p]]) for the gate|up GEMMs' TMA boxes.
+cudaError_t launch_gather_rows(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
+                               const int32_t* sorted_token, cudaStream_t st);
+
+// The same grouped GEMMs on CTA pairs (tcgen05.mma.cta_group::2, M = 256): each SM holds
+// half of a token tile, and the down GEMM takes the hi and lo halves of h in one MMA.
+// For batches with many tokens per expert (prefill).
+cudaError_t launch_tc2_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
+                               const int32_t* sorted_token, const moe_weights& w, cudaStream_t st);
+cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
+                            const int32_t* sorted_token, const float* sorted_w, const float* sgate,
+                            const moe_weights& w, float* y, float* y_shared, float* out,
+                            cudaStream_t st);
+
 }  // namespace moe

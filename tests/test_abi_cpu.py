@@ -102,7 +102,7 @@ def test_empty_batch_is_a_no_op():
 
 def test_variant_setter():
     assert moe.lib().moe_set_variant(7) == moe.MOE_ERR_INVALID_ARG
-    for v in (moe.MOE_VARIANT_STREAM, moe.MOE_VARIANT_TC, moe.MOE_VARIANT_AUTO):
+    for v in (moe.MOE_VARIANT_STREAM, moe.MOE_VARIANT_TC, moe.MOE_VARIANT_TC2, moe.MOE_VARIANT_AUTO):
         moe.moe_set_variant(v)
 
 

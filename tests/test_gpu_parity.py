@@ -18,7 +18,7 @@ import sparse_moe_expert_fp32_b200 as moe  # noqa: E402
 import synth  # noqa: E402
 from parity_util import NEAR_TIE_GAP, assert_layer_close, err_stats, id_sets_match  # noqa: E402
 
-VARIANTS = {"stream": moe.MOE_VARIANT_STREAM, "tc": moe.MOE_VARIANT_TC}
+VARIANTS = {"stream": moe.MOE_VARIANT_STREAM, "tc": moe.MOE_VARIANT_TC, "tc2": moe.MOE_VARIANT_TC2}
 
 
 def _u16(t):
