@@ -290,6 +290,19 @@ def run_ours(args, cfg, world, rank, local):
                "tc": moe.MOE_VARIANT_TC, "tc2": moe.MOE_VARIANT_TC2}[args.variant]
     moe.moe_set_variant(variant)
     dev = synth.device_inputs(cfg, seed=0, x_seed=rank, device=f"cuda:{local}")
+    compact = None
+    if args.compact:
+        # weight pre-pass (once, at load time): drop zero gate/up channels and their down
+        # columns; the layer then runs with I = I_c
+        full_cfg = cfg
+        t0 = time.time()
+        dev, I_c = moe.compact_zero_channels(moe.shape_of(cfg), dev)
+        torch.cuda.synchronize()
+        compact = {"I": cfg.I, "I_c": I_c, "prepass_s": round(time.time() - t0, 3),
+                   "dense_equivalent_flops": 6.0 * (full_cfg.R * full_cfg.H * full_cfg.I
+                                                    + full_cfg.T * full_cfg.H * full_cfg.Is)}
+        cfg = cfg.replace(I=I_c)
+        torch.cuda.empty_cache()
     s = moe.shape_of(cfg)
     ws = moe.alloc_workspace(s, host_staging=True)
     out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
@@ -429,6 +442,7 @@ def run_ours(args, cfg, world, rank, local):
             "config": config_block(cfg, args.variant,
                                    "host launches of one layer forward per step" if args.no_graph
                                    else "CUDA graph replay of one layer forward per step"),
+            "zero_channel_compaction": compact,
             "roofline": roofline,
             "graph": not args.no_graph,
             "e2e": {"value": cfg.T * args.steps * world / (ms_e2e / 1e3), "unit": "tokens/s",
@@ -436,7 +450,7 @@ def run_ours(args, cfg, world, rank, local):
             "gpu_launches": launches, "kernels": kernels,
             "clocks": sampler.summary(windows) if sampler else None}
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg)
+        line["cpu_baseline"] = cpu_baseline(full_cfg if compact else cfg)
     return line
 
 
@@ -452,6 +466,8 @@ def main():
     ap.add_argument("--variant", default="auto", choices=["auto", "stream", "tc", "tc2"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel from the host")
+    ap.add_argument("--compact", action="store_true",
+                    help="zero-channel compaction of the routed experts before timing (weight pre-pass)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = synth.CONFIGS[args.workload]

@@ -202,6 +202,42 @@ moe_status moe_layer_forward_host(const moe_shape* shape, const void* x_host,
                                   const moe_weights* weights, float* out_host, void* ws,
                                   size_t ws_bytes, void* stream);
 
+/*
+ * Zero-channel compaction of structurally sparse routed experts: a weight pre-pass run once
+ * when the weights are loaded, not a step of the layer.
+ * Source: "Qwen3.8-2.4T-A95B" discussion #29, tensor table. The GGUF zero fractions show
+ * 71.0 % of the ffn_gate_exps and ffn_up_exps rows of a 2.4T layer as exact zeros.
+ * Channel c of routed expert e is dead when gate row W_gate,e[c,:] or up row W_up,e[c,:]
+ * is all zero (every bf16 element +0 or -0). Then h_c = SiLU(g_c) * u_c = 0 exactly, and
+ * down column c adds nothing to expert(x) = W_down (SiLU(W_gate x) * W_up x).
+ * Compaction keeps each expert's live channels in their original order, packed to the
+ * front of a common width I_c, with zeros after them. The layer then runs on the
+ * compacted bank with moe_shape.I = I_c. Its outputs are those of the full bank up to
+ * the order of fp32 additions. Gate/up/down bytes and FLOPs scale by I_c / I.
+ * The shared expert is not touched.
+ *
+ * moe_compact_workspace_bytes: scratch size for the two calls below (caller-owned device
+ *   memory, 16-byte aligned; about 5*E*I + 4*E bytes). 0 for an invalid shape.
+ * moe_zero_channel_count: scans w_gate_up (bf16 [E][2I][H]) and writes to *max_live (host
+ *   int32) the largest live-channel count of any expert. It SYNCHRONISES `stream` (the
+ *   count is read back); do not call it inside a stream capture.
+ * moe_compact_zero_channels: writes gate_up_c (bf16 [E][2*I_c][H], rows 0..I_c-1 gate,
+ *   I_c..2*I_c-1 up) and down_c (bf16 [E][H][I_c]) from w_gate_up and w_down (bf16
+ *   [E][H][I]); asynchronous on `stream`. I_c must be a multiple of 64, at most I, and at
+ *   least the count from moe_zero_channel_count. The tensor-core layer kernels also need a
+ *   multiple of 128, so round the count up to 128. If some expert has more live channels
+ *   than I_c, its extra channels are dropped and the bounds flag is set in the
+ *   workspace's status word; moe_device_status(ws, ...) reports it as
+ *   MOE_ERR_DEVICE_BOUNDS. Errors: MOE_ERR_INVALID_ARG (null or misaligned pointer, bad
+ *   I_c), MOE_ERR_WORKSPACE_TOO_SMALL, MOE_ERR_CUDA.
+ */
+size_t moe_compact_workspace_bytes(const moe_shape* shape);
+moe_status moe_zero_channel_count(const moe_shape* shape, const void* w_gate_up,
+                                  int32_t* max_live, void* ws, size_t ws_bytes, void* stream);
+moe_status moe_compact_zero_channels(const moe_shape* shape, const void* w_gate_up,
+                                     const void* w_down, int32_t I_c, void* gate_up_c,
+                                     void* down_c, void* ws, size_t ws_bytes, void* stream);
+
 /* Choose the grouped-GEMM variant for later calls (process-wide; default AUTO). */
 moe_status moe_set_variant(moe_variant variant);
 

@@ -75,6 +75,9 @@ _SIGS = {
     "moe_layer_forward": ([_SP, _vp, _WP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_layer_forward_host": ([_SP, _vp, _WP, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_set_variant": ([ctypes.c_int], ctypes.c_int),
+    "moe_compact_workspace_bytes": ([_SP], _sz),
+    "moe_zero_channel_count": ([_SP, _vp, ctypes.POINTER(ctypes.c_int32), _vp, _sz, _vp], ctypes.c_int),
+    "moe_compact_zero_channels": ([_SP, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_device_status": ([_vp, _sz, _vp, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
     "moe_debug_wait_flag": ([_vp, _u64, _vp, _sz, _vp], ctypes.c_int),
     "moe_profile_enable": ([_i32], ctypes.c_int),
@@ -213,6 +216,29 @@ def moe_layer_forward_host(shape, x_host, weights, out_host, ws, stream=None):
            "moe_layer_forward_host")
 
 
+def moe_compact_workspace_bytes(shape: moe_shape) -> int:
+    n = _lib.moe_compact_workspace_bytes(ctypes.byref(shape))
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_compact_workspace_bytes")
+    return n
+
+
+def moe_zero_channel_count(shape, w_gate_up, ws, stream=None) -> int:
+    """Largest number of live channels of any routed expert (synchronises the stream)."""
+    m = ctypes.c_int32(0)
+    _check(_lib.moe_zero_channel_count(ctypes.byref(shape), _ptr(w_gate_up), ctypes.byref(m),
+                                       _ptr(ws), _nbytes(ws), _stream(stream)),
+           "moe_zero_channel_count")
+    return int(m.value)
+
+
+def moe_compact_zero_channels(shape, w_gate_up, w_down, I_c, gate_up_c, down_c, ws, stream=None):
+    _check(_lib.moe_compact_zero_channels(ctypes.byref(shape), _ptr(w_gate_up), _ptr(w_down),
+                                          int(I_c), _ptr(gate_up_c), _ptr(down_c), _ptr(ws),
+                                          _nbytes(ws), _stream(stream)),
+           "moe_compact_zero_channels")
+
+
 def moe_set_variant(variant: int) -> None:
     _check(_lib.moe_set_variant(int(variant)), "moe_set_variant")
 
@@ -255,3 +281,29 @@ def alloc_workspace(shape: moe_shape, device="cuda", host_staging: bool = False,
     ws = torch.empty(n, dtype=torch.uint8, device=device)
     moe_workspace_init(ws, stream)
     return ws
+
+
+def compact_zero_channels(shape: moe_shape, weights: dict, multiple: int = 128, stream=None):
+    """Zero-channel compaction of a weight dict (the pre-pass, run once).
+
+    Returns (new weight dict sharing every tensor but the routed banks, I_c), with I_c the
+    largest live-channel count rounded up to `multiple` (128 suits the tensor-core
+    kernels). Run the layer on the result with moe_shape.I = I_c. Raises if a device
+    check fails.
+    """
+    import torch
+
+    ws = torch.empty(moe_compact_workspace_bytes(shape), dtype=torch.uint8,
+                     device=weights["w_gate_up"].device)
+    m = moe_zero_channel_count(shape, weights["w_gate_up"], ws, stream)
+    I_c = min(shape.I, max(multiple, -(-m // multiple) * multiple))
+    E, H = shape.E, shape.H
+    gu = torch.empty((E, 2 * I_c, H), dtype=weights["w_gate_up"].dtype, device=ws.device)
+    dn = torch.empty((E, H, I_c), dtype=weights["w_down"].dtype, device=ws.device)
+    moe_compact_zero_channels(shape, weights["w_gate_up"], weights["w_down"], I_c, gu, dn, ws, stream)
+    st, flags = moe_device_status(ws, stream)
+    _check(st, "moe_compact_zero_channels (device)")
+    out = dict(weights)
+    out["w_gate_up"] = gu
+    out["w_down"] = dn
+    return out, I_c

@@ -335,6 +335,56 @@ moe_status moe_layer_forward_host(const moe_shape* shape, const void* x_host,
   return MOE_OK;
 }
 
+size_t moe_compact_workspace_bytes(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return compact_workspace_bytes(*shape);
+}
+
+moe_status moe_zero_channel_count(const moe_shape* shape, const void* w_gate_up,
+                                  int32_t* max_live, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_shape(shape));
+  const moe_shape& s = *shape;
+  if (!aligned16(w_gate_up) || !max_live || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < compact_workspace_bytes(s)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* w = static_cast<char*>(ws);
+  MOE_CUDA(cudaMemsetAsync(w, 0, 256, st));
+  int32_t *src = nullptr, *count = nullptr;
+  MOE_CUDA(launch_zero_channel_map(s, static_cast<const uint16_t*>(w_gate_up), s.I, w, &src,
+                                   &count, st));
+  std::vector<int32_t> counts((size_t)s.E);
+  MOE_CUDA(cudaMemcpyAsync(counts.data(), count, counts.size() * sizeof(int32_t),
+                           cudaMemcpyDeviceToHost, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  int32_t m = 0;
+  for (int32_t c : counts) m = c > m ? c : m;
+  *max_live = m;
+  return MOE_OK;
+}
+
+moe_status moe_compact_zero_channels(const moe_shape* shape, const void* w_gate_up,
+                                     const void* w_down, int32_t I_c, void* gate_up_c,
+                                     void* down_c, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_shape(shape));
+  const moe_shape& s = *shape;
+  if (!aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(gate_up_c) ||
+      !aligned16(down_c) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  if (I_c <= 0 || I_c % 64 || I_c > s.I) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < compact_workspace_bytes(s)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* w = static_cast<char*>(ws);
+  MOE_CUDA(cudaMemsetAsync(w, 0, 256, st));
+  int32_t *src = nullptr, *count = nullptr;
+  MOE_CUDA(launch_zero_channel_map(s, static_cast<const uint16_t*>(w_gate_up), I_c, w, &src,
+                                   &count, st));
+  MOE_CUDA(launch_compact_banks(s, static_cast<const uint16_t*>(w_gate_up),
+                                static_cast<const uint16_t*>(w_down), src, I_c,
+                                static_cast<uint16_t*>(gate_up_c), static_cast<uint16_t*>(down_c),
+                                st));
+  return MOE_OK;
+}
+
 moe_status moe_set_variant(moe_variant variant) {
   if (variant != MOE_VARIANT_AUTO && variant != MOE_VARIANT_STREAM && variant != MOE_VARIANT_TC &&
       variant != MOE_VARIANT_TC2)

@@ -115,6 +115,13 @@ cudaError_t launch_stream_down(const moe_shape& s, const Layout& L, char* ws,
 cudaError_t launch_combine(const moe_shape& s, const float* y, const float* y_shared,
                            const int32_t* assign_row, const float* topk_w, const float* sgate,
                            float* out, cudaStream_t st);
+// Zero-channel compaction (a weight pre-pass; compact.cu).
+size_t compact_workspace_bytes(const moe_shape& s);
+cudaError_t launch_zero_channel_map(const moe_shape& s, const uint16_t* w_gate_up, int Ic,
+                                    char* ws, int32_t** src, int32_t** count, cudaStream_t st);
+cudaError_t launch_compact_banks(const moe_shape& s, const uint16_t* w_gate_up,
+                                 const uint16_t* w_down, const int32_t* src, int Ic,
+                                 uint16_t* gate_up_c, uint16_t* down_c, cudaStream_t st);
 cudaError_t launch_wait_flag(const int32_t* flag, uint64_t timeout_ns, uint32_t* status,
                              cudaStream_t st);
 

@@ -339,6 +339,53 @@ def pin_zero_channels_delete():
     assert np.isfinite(r["out"]).all()
 
 
+def pin_zero_channel_rule():
+    """A channel dies if its gate row OR its up row is all +-0; one nonzero value keeps it."""
+    rng = np.random.default_rng(21)
+    inp = _tiny_inputs(rng, T=7, H=16, E=3, k=2, I=6, Is=4)
+    gu = inp["w_gate_up"].copy()
+    I = 6
+    gu[0, 1] = 0                       # gate row only
+    gu[0, I + 3] = 0                   # up row only
+    gu[1, 2] = 0x8000                  # gate row of -0.0
+    gu[1, I + 2] = 0                   # and its up row
+    gu[2, 4] = 0
+    gu[2, 4, 7] = 0x3F80               # one 1.0 left: live
+    gu[2, I + 5] = 0x8000              # up row of -0.0
+    live = [oracle.live_channels(gu[e]).tolist() for e in range(3)]
+    assert live[0] == [True, False, True, False, True, True]
+    assert live[1] == [True, True, False, True, True, True]
+    assert live[2] == [True, True, True, True, True, False]
+
+
+def pin_compaction_keeps_the_layer():
+    """The layer on the compacted bank (I -> I_c) equals the layer on the full bank."""
+    cfg = synth.LayerConfig("z", T=9, H=32, E=5, k=2, I=16, Is=16, zero_rows_pct=50)
+    h = synth.host_inputs(cfg, seed=22)
+    gu, d = h.gate_up_all(), h.down_all()
+    gu[3, 2] = 0  # one more dead channel, by its gate row only
+    n_live = max(int(oracle.live_channels(gu[e]).sum()) for e in range(cfg.E))
+    assert n_live == 8
+    gu_c, d_c = oracle.compact_zero_channels(gu, d, 8)
+    full = oracle.moe_forward(h.x, h.w_router, None, gu, d, h.ws_gate_up, h.ws_down,
+                              h.w_shared_gate, cfg.k)
+    comp = oracle.moe_forward(h.x, h.w_router, None, gu_c, d_c, h.ws_gate_up, h.ws_down,
+                              h.w_shared_gate, cfg.k)
+    assert (full["ids"] == comp["ids"]).all()
+    assert np.allclose(comp["out"], full["out"], rtol=1e-12, atol=1e-15)
+    # live channels in their original order, then zero padding
+    keep = np.nonzero(oracle.live_channels(gu[3]))[0]
+    assert (gu_c[3, :keep.size] == gu[3, keep]).all() and (gu_c[3, keep.size:8] == 0).all()
+    assert (d_c[3][:, :keep.size] == d[3][:, keep]).all() and (d_c[3][:, keep.size:] == 0).all()
+    # wider padding changes nothing; too narrow is refused
+    gu_w, d_w = oracle.compact_zero_channels(gu, d, 12)
+    wide = oracle.moe_forward(h.x, h.w_router, None, gu_w, d_w, h.ws_gate_up, h.ws_down,
+                              h.w_shared_gate, cfg.k)
+    assert np.allclose(wide["out"], full["out"], rtol=1e-12, atol=1e-15)
+    with pytest.raises(ValueError):
+        oracle.compact_zero_channels(gu, d, 7)
+
+
 def pin_permute():
     rng = np.random.default_rng(13)
     T, E, k = 37, 9, 4
@@ -367,7 +414,8 @@ PINS = [pin_page_counts, pin_zero_fraction, pin_bf16_decoding, pin_silu_closed_f
         pin_routing_weights, pin_topk_order_and_ties, pin_forced_expert_is_dense_swiglu,
         pin_all_experts_is_softmax_mixture, pin_shared_gate_half, pin_brute_force_tiny,
         pin_brute_force_generator_inputs, pin_expert_relabelling, pin_token_independence,
-        pin_zero_channels_delete, pin_permute, pin_packed_outputs_and_combine]
+        pin_zero_channels_delete, pin_zero_channel_rule, pin_compaction_keeps_the_layer,
+        pin_permute, pin_packed_outputs_and_combine]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -427,9 +475,24 @@ def _mut_permute_unstable(ids, E):
     return off, st, ar, slot
 
 
+def _mut_zero_rule_gate_only(w_gate_up_e):
+    w = moe_oracle.bf16_to_f64(w_gate_up_e)
+    return (w[: w.shape[0] // 2] != 0.0).any(axis=1)
+
+
+def _mut_compaction_down_misaligned(w_gate_up, w_down, I_c):
+    gu, dn = _ORIG["compact_zero_channels"](w_gate_up, w_down, I_c)
+    return gu, np.roll(dn, 1, axis=2)  # down columns one channel off
+
+
+def _mut_compaction_reversed(w_gate_up, w_down, I_c):
+    gu, dn = _ORIG["compact_zero_channels"](w_gate_up, w_down, I_c)
+    return gu[:, ::-1].copy(), dn[:, :, ::-1].copy()  # consistent, but not the specified order
+
+
 _ORIG = {n: getattr(moe_oracle, n) for n in
          ("silu", "shared_gate", "routing_weights", "swiglu_expert", "topk_select", "router_logits",
-          "permute")}
+          "permute", "compact_zero_channels")}
 
 MUTATIONS = {
     "silu_sign": ("silu", _mut_silu_sign),
@@ -440,6 +503,9 @@ MUTATIONS = {
     "router_bias_ignored": ("router_logits", _mut_bias_ignored),
     "softmax_sign": ("routing_weights", _mut_softmax_wrong_sign),
     "unstable_dispatch": ("permute", _mut_permute_unstable),
+    "zero_rule_gate_only": ("live_channels", _mut_zero_rule_gate_only),
+    "compaction_down_misaligned": ("compact_zero_channels", _mut_compaction_down_misaligned),
+    "compaction_reversed": ("compact_zero_channels", _mut_compaction_reversed),
 }
 
 
