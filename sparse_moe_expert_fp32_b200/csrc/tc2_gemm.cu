@@ -246,8 +246,13 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   } else if (warp == 1) {
     // ------------------------------------------------------------ pair MMA issuer (leader)
     if (rank == 0 && lane == 0) {
-      int it = 0, nt = 0;
+      // Kept short on purpose: the tensor core takes an MMA only about when it can start
+      // it, so every instruction between a stage's MMAs and the next stage's is idle time
+      // for it (running ring position instead of division, one asm block per stage).
+      int s = 0, nt = 0;
+      uint32_t ph = 0;
       bool aborted = false;
+      const uint64_t desc0 = ptx::smem_desc_kmajor<kRowB>(smem);  // stage 0, A operand
       for (int tile = pair; tile < total && !aborted; tile += npairs, ++nt) {
         const PairGeom G = pair_geom<MODE>(args, S, tile, R, rank, plane_rows);
         const int slot = nt & 1;
@@ -259,23 +264,20 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         ptx::tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(slot * kSlotCols);
         const uint32_t idesc = ptx::idesc_bf16_f32(256, G.n_mma);
-        for (int ks = 0; ks < G.nk; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          // The copies' completion on the full barrier orders them before the MMAs that read
-          // the stage; no tcgen05 fence is needed here (one per stage serialised the MMAs).
-          // A non-blocking test first: a stage that has landed costs no suspended wait.
-          if (!ptx::mbar_test_wait(&S.full[s], ph) && !wait_phase(&S.full[s], ph, S, args.status)) {
+        for (int ks = 0; ks < G.nk; ++ks) {
+          // The copies' completion on the full barrier orders them before the MMAs that
+          // read the stage; no tcgen05 fence is needed here.
+          if (!wait_phase(&S.full[s], ph, S, args.status)) {
             aborted = true;
             break;
           }
-          const uint8_t* st = smem + s * kStageBytes;
-          const uint64_t ad = ptx::smem_desc_kmajor<kRowB>(st);
-          const uint64_t bd = ptx::smem_desc_kmajor<kRowB>(st + kABytes);
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes along K = +2 in the address field
-            ptx::umma_bf16_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t ad = desc0 + (uint64_t)s * (kStageBytes >> 4);
+          ptx::umma_bf16_pair_x4(d, ad, ad + (kABytes >> 4), idesc, ks > 0 ? 1u : 0u);
           ptx::umma_commit_pair(&S.empty[s], 0x3);
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
         if (aborted) break;
         ptx::umma_commit_pair(&S.tmem_full[slot], 0x3);

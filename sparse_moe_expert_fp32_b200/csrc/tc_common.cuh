@@ -67,11 +67,12 @@ __device__ __forceinline__ Tile decode_tile(const int* row0, const int* tp, int 
 }
 
 // Bounded wait on an mbarrier phase; false if it ran out (flag recorded) or another role
-// already gave up.
+// already gave up. The fast path is one non-blocking test (a blocking try_wait costs ~170
+// cycles even on a completed phase, idle time for the tensor core when the MMA-issuing
+// thread pays it); the waiting loop is out of line so that the issue loops stay short.
 template <class State>
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, State& S,
-                                           uint32_t* status) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_phase_slow(uint64_t* bar, uint32_t parity, State& S,
+                                             uint32_t* status) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
@@ -84,6 +85,13 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, State
       }
     }
   }
+}
+
+template <class State>
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, State& S,
+                                           uint32_t* status) {
+  if (ptx::mbar_test_wait(bar, parity)) return true;
+  return wait_phase_slow(bar, parity, S, status);
 }
 
 // Short bounded wait used while leaving after an abort.

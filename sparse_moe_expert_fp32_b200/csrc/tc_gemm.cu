@@ -331,9 +331,15 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int it = 0;
+      // Kept short on purpose: the tensor core takes an MMA only about when it can start
+      // it, so every instruction between MMAs is idle time for it (running ring position,
+      // four MMAs per asm block).
+      int s = 0;
+      uint32_t ph = 0;
       Slots sl;
       bool aborted = false;
+      const uint64_t desc0 = ptx::smem_desc_kmajor<C::kRowBytes>(smem);  // stage 0, first A tile
+      constexpr uint64_t kDA = C::kATileBytes >> 4, kDB = C::kBTileBytes >> 4;
       for (int qi = 0; !aborted; ++qi) {
         const int slot = qi % kQueue;
         if (!wait_phase(&S.q_full[slot], (uint32_t)(qi / kQueue) & 1u, S, args.status)) {
@@ -356,33 +362,27 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         ptx::tc_fence_after();
         const uint32_t d0 = tmem + first * kSlotCols;
         const uint32_t d1 = d0 + (count == 2 ? kSlotCols : 128u);
-        for (int ks = 0; ks < G.nk; ++ks, ++it) {
-          const int s = it % C::kStages;
-          const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
-          // The copies' completion on the full barrier orders them before the MMAs that read
-          // the stage; no tcgen05 fence is needed here (one per stage serialised the MMAs).
-          // A non-blocking test first: a stage that has landed costs no suspended wait.
-          if (!ptx::mbar_test_wait(&S.full[s], ph) && !wait_phase(&S.full[s], ph, S, args.status)) {
+        for (int ks = 0; ks < G.nk; ++ks) {
+          // The copies' completion on the full barrier orders them before the MMAs that
+          // read the stage; no tcgen05 fence is needed here.
+          if (!wait_phase(&S.full[s], ph, S, args.status)) {
             aborted = true;
             break;
           }
-          const uint8_t* st = smem + s * C::kStageBytes;
-          const uint64_t a0 = ptx::smem_desc_kmajor<C::kRowBytes>(st);
-          const uint64_t a1 = ptx::smem_desc_kmajor<C::kRowBytes>(st + C::kATileBytes);
-          const uint64_t bd = ptx::smem_desc_kmajor<C::kRowBytes>(st + 2 * C::kATileBytes);
-#pragma unroll
-          for (int kk = 0; kk < C::kKK; ++kk) {
-            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-            // +32 bytes along K inside the swizzle atom = +2 in the address field
-            ptx::umma_bf16(d0, a0 + 2 * kk, bd + 2 * kk, idesc, acc);
-            ptx::umma_bf16(d1, a1 + 2 * kk, bd + 2 * kk, idesc, acc);
-            if (MODE == kDown) {  // the lo half of h into the same accumulators
-              const uint64_t bl = bd + (C::kBTileBytes >> 4);
-              ptx::umma_bf16(d0, a0 + 2 * kk, bl + 2 * kk, idesc, 1u);
-              ptx::umma_bf16(d1, a1 + 2 * kk, bl + 2 * kk, idesc, 1u);
-            }
+          const uint64_t a0 = desc0 + (uint64_t)s * (C::kStageBytes >> 4);
+          const uint64_t bd = a0 + 2 * kDA;
+          const uint32_t acc = ks > 0 ? 1u : 0u;
+          ptx::umma_bf16_x4(d0, a0, bd, idesc, acc);
+          ptx::umma_bf16_x4(d1, a0 + kDA, bd, idesc, acc);
+          if (MODE == kDown) {  // the lo half of h into the same accumulators
+            ptx::umma_bf16_x4(d0, a0, bd + kDB, idesc, 1u);
+            ptx::umma_bf16_x4(d1, a0 + kDA, bd + kDB, idesc, 1u);
           }
           ptx::umma_commit(&S.empty[s]);
+          if (++s == C::kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
         if (aborted) break;
         for (int i = 0; i < count; ++i) ptx::umma_commit(&S.tmem_full[(first + i) & 1]);
