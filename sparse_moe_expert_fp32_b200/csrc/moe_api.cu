@@ -150,18 +150,11 @@ bool use_tc(const moe_shape& s) {
   return tc_supported(s);
 }
 
-// CTA-pair kernels for this shape (gate|up and down decided separately)? They pay off once
-// the token tiles are wide: AUTO takes them when the batch averages at least 16 routed rows
-// per expert, except the gate|up GEMM at hidden sizes above 4096, where its 128-stage K loop
-// ran faster on the one-CTA kernel (B200, 2.4T-shaped prefill: 6.82 ms against 7.70 ms; at
-// hidden 2560 the pair kernel wins, 0.71 ms against 0.77 ms).
-bool use_tc2_gate_up(const moe_shape& s) {
-  const int v = g_variant.load();
-  if (v == MOE_VARIANT_TC2) return true;
-  return v == MOE_VARIANT_AUTO && (int64_t)s.T * s.k >= 16 * (int64_t)s.E && s.H <= 4096;
-}
-
-bool use_tc2_down(const moe_shape& s) {
+// CTA-pair kernels for this shape? They pay off once the token tiles are wide: AUTO takes
+// them when the batch averages at least 16 routed rows per expert (B200: 2.4T-shaped
+// prefill gate|up 6.92 ms against 6.99, down 6.94 against 8.00; Flash-Next-shaped prefill
+// gate|up 0.71 against 0.78; at decode sizes the one-CTA kernels' 16-token tiles suffice).
+bool use_tc2(const moe_shape& s) {
   const int v = g_variant.load();
   if (v == MOE_VARIANT_TC2) return true;
   return v == MOE_VARIANT_AUTO && (int64_t)s.T * s.k >= 16 * (int64_t)s.E;
@@ -173,12 +166,13 @@ moe_status run_grouped(const moe_shape& s, const Layout& L, char* ws, const uint
                        const moe_weights& w, float* y, float* y_shared, float* out,
                        cudaStream_t st) {
   if (use_tc(s)) {
-    if (use_tc2_gate_up(s)) MOE_CUDA(launch_tc2_gate_up(s, L, ws, x, sorted_token, w, st));
-    else MOE_CUDA(launch_tc_gate_up(s, L, ws, x, sorted_token, w, st));
-    if (use_tc2_down(s))
+    if (use_tc2(s)) {
+      MOE_CUDA(launch_tc2_gate_up(s, L, ws, x, sorted_token, w, st));
       MOE_CUDA(launch_tc2_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));
-    else
+    } else {
+      MOE_CUDA(launch_tc_gate_up(s, L, ws, x, sorted_token, w, st));
       MOE_CUDA(launch_tc_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));
+    }
   } else {
     MOE_CUDA(launch_stream_gate_up(s, L, ws, x, sorted_token, w, st));
     MOE_CUDA(launch_stream_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));

@@ -41,12 +41,25 @@ namespace {
 
 constexpr int kEpi = 8;
 constexpr int kThreads2 = 64 + 32 * kEpi;
-constexpr int kBK = 64;                       // K per stage: 128-byte rows, 128-byte swizzle
-constexpr uint32_t kRowB = kBK * 2;
-constexpr uint32_t kABytes = 128u * kRowB;    // this CTA's 128 weight rows
-constexpr uint32_t kBBytes = 128u * kRowB;    // this CTA's token half, at most 128 rows
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr int kStages = 6;
+// A stage holds KSUB sub-tiles of 64 K of both operands (128-byte rows, 128-byte swizzle,
+// the widest a TMA box may be). With KSUB = 2, eight MMAs share one hand-off (wait, commit)
+// between the producer and the MMA issuer, which paid off on long K loops (hidden 8192;
+// inter 2048) and cost on short ones (inter 640: 5 stages per tile), where KSUB = 1 keeps a
+// 6-deep ring.
+constexpr int kBK = 64;                   // K per sub-tile
+constexpr uint32_t kRowB = kBK * 2;       // bytes per sub-tile row
+constexpr uint32_t kASub = 128u * kRowB;  // 128 weight rows of one sub-tile: 16 KB
+constexpr uint32_t kBSub = 128u * kRowB;  // up to 128 token rows of one sub-tile
+
+template <int KSUB>
+struct Ring {
+  static constexpr int kStageK = kBK * KSUB;                   // K per stage
+  static constexpr uint32_t kABytes = KSUB * kASub;            // this CTA's weight rows
+  static constexpr uint32_t kBBytes = KSUB * kBSub;            // this CTA's token half
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;   // 32 or 64 KB
+  static constexpr int kStages = KSUB == 1 ? 6 : 3;
+};
+constexpr int kMaxStages = 6;
 constexpr int kSlotCols = 256;
 constexpr int kBoxes = 5;  // token boxes of 128, 64, 32, 16 and 8 rows
 __host__ __device__ constexpr int box_rows(int i) { return 128 >> i; }
@@ -54,8 +67,8 @@ __host__ __device__ constexpr int box_rows(int i) { return 128 >> i; }
 enum PairMode { kPairGateUp = 0, kPairDown = 1 };
 
 struct PairShared {
-  uint64_t full[kStages];   // leader: both CTAs' copies of a stage have landed
-  uint64_t empty[kStages];  // each CTA: the MMAs reading its copy of a stage are done
+  uint64_t full[kMaxStages];   // leader: both CTAs' copies of a stage have landed
+  uint64_t empty[kMaxStages];  // each CTA: the MMAs reading its copy of a stage are done
   uint64_t tmem_full[2];    // each CTA: the accumulator slot holds a finished tile
   uint64_t tmem_empty[2];   // leader: both CTAs' epilogues have drained the slot
   uint64_t drain;
@@ -69,10 +82,12 @@ struct PairShared {
   };
 };
 
+template <int KSUB>
 constexpr size_t pair_smem_bytes() {
-  return 1024 + (size_t)kStages * kStageBytes + sizeof(PairShared);
+  return 1024 + (size_t)Ring<KSUB>::kStages * Ring<KSUB>::kStageBytes + sizeof(PairShared);
 }
-static_assert(pair_smem_bytes() <= 232448, "over the 227 KB of shared memory a CTA may use");
+static_assert(pair_smem_bytes<1>() <= 232448 && pair_smem_bytes<2>() <= 232448,
+              "over the 227 KB of shared memory a CTA may use");
 
 struct PairMaps {
   CUtensorMap m[kBoxes];
@@ -107,9 +122,10 @@ struct PairGeom {
   bool shared;
 };
 
-template <int MODE>
+template <int MODE, int KSUB>
 __device__ __forceinline__ PairGeom pair_geom(const TcArgs& a, const PairShared& S, int tile,
                                               int R, int rank, int plane_rows) {
+  constexpr int kStageK = Ring<KSUB>::kStageK;
   PairGeom G;
   G.t = decode_tile(S.row0, S.tp, a.E, tile, MODE == kPairGateUp ? 256 : 128);
   G.shared = G.t.g == a.E;
@@ -121,7 +137,7 @@ __device__ __forceinline__ PairGeom pair_geom(const TcArgs& a, const PairShared&
     G.nb = G.t.N / 2;
     G.b_row = (G.shared ? G.t.p0 - R : G.t.p0) + rank * G.nb;
     G.n_mma = G.t.N;
-    G.nk = a.H / kBK;
+    G.nk = a.H / kStageK;
   } else {
     const int base = G.shared ? 0 : G.t.g * a.H;
     G.a_row0 = base + G.t.m * 256 + rank * 128;
@@ -129,16 +145,19 @@ __device__ __forceinline__ PairGeom pair_geom(const TcArgs& a, const PairShared&
     G.nb = G.t.N;
     G.b_row = G.t.p0 + rank * plane_rows;
     G.n_mma = 2 * G.t.N;
-    G.nk = (G.shared ? a.Is : a.I) / kBK;
+    G.nk = (G.shared ? a.Is : a.I) / kStageK;
   }
   return G;
 }
 
-template <int MODE>
+template <int MODE, int KSUB>
 __global__ void __launch_bounds__(kThreads2, 1)
 tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_sh,
                    const __grid_constant__ PairMaps tm_b, const __grid_constant__ PairMaps tm_b_sh,
                    const TcArgs args) {
+  using RG = Ring<KSUB>;
+  constexpr int kStages = RG::kStages, kStageK = RG::kStageK;
+  constexpr uint32_t kABytes = RG::kABytes, kStageBytes = RG::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -195,13 +214,13 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     int it = 0;
     bool aborted = false;
     for (int tile = pair; tile < total && !aborted; tile += npairs) {
-      const PairGeom G = pair_geom<MODE>(args, S, tile, R, rank, plane_rows);
+      const PairGeom G = pair_geom<MODE, KSUB>(args, S, tile, R, rank, plane_rows);
       const CUtensorMap* my_map = nullptr;
       uint32_t my_off = 0;
       int my_row = 0;
       if (MODE == kPairGateUp && lane < 2) {  // 64 gate rows, then 64 up rows
         my_map = G.shared ? &tm_a_sh : &tm_a;
-        my_off = lane * (kABytes / 2);
+        my_off = lane * (kASub / 2);
         my_row = lane ? G.a_row1 : G.a_row0;
       } else if (MODE == kPairDown && lane == 0) {
         my_map = G.shared ? &tm_a_sh : &tm_a;
@@ -211,11 +230,11 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         if (b_piece(G.nb, lane - 2, r, bi)) {
           const PairMaps& bm = (MODE == kPairGateUp && G.shared) ? tm_b_sh : tm_b;
           my_map = &bm.m[bi];
-          my_off = kABytes + (uint32_t)r * kRowB;
+          my_off = kABytes + (uint32_t)r * kRowB;  // sub-tile j adds j * kBSub
           my_row = G.b_row + r;
         }
       }
-      const uint32_t bytes = 2u * (kABytes + (uint32_t)G.nb * kRowB);  // both CTAs
+      const uint32_t bytes = 2u * KSUB * (kASub + (uint32_t)G.nb * kRowB);  // both CTAs
       for (int ks = 0; ks < G.nk; ++ks, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -229,8 +248,11 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           break;
         }
         if (my_map)
-          ptx::tma_load_2d_pair(smem + s * kStageBytes + my_off, my_map,
-                                full0 + (uint32_t)(s * sizeof(uint64_t)), ks * kBK, my_row);
+#pragma unroll
+          for (int j = 0; j < KSUB; ++j)  // weight sub-tiles at j * kASub, token ones at j * kBSub
+            ptx::tma_load_2d_pair(smem + s * kStageBytes + my_off + j * (my_off < kABytes ? kASub : kBSub),
+                                  my_map, full0 + (uint32_t)(s * sizeof(uint64_t)),
+                                  ks * kStageK + j * kBK, my_row);
       }
     }
     // wait until the MMAs have released every stage this CTA filled, so that no commit
@@ -254,7 +276,7 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       bool aborted = false;
       const uint64_t desc0 = ptx::smem_desc_kmajor<kRowB>(smem);  // stage 0, A operand
       for (int tile = pair; tile < total && !aborted; tile += npairs, ++nt) {
-        const PairGeom G = pair_geom<MODE>(args, S, tile, R, rank, plane_rows);
+        const PairGeom G = pair_geom<MODE, KSUB>(args, S, tile, R, rank, plane_rows);
         const int slot = nt & 1;
         const uint32_t use = (uint32_t)(nt >> 1);
         if (!wait_phase(&S.tmem_empty[slot], (use & 1u) ^ 1u, S, args.status)) {
@@ -273,6 +295,8 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           }
           const uint64_t ad = desc0 + (uint64_t)s * (kStageBytes >> 4);
           ptx::umma_bf16_pair_x4(d, ad, ad + (kABytes >> 4), idesc, ks > 0 ? 1u : 0u);
+          if (KSUB == 2)
+            ptx::umma_bf16_pair_x4(d, ad + (kASub >> 4), ad + ((kABytes + kBSub) >> 4), idesc, 1u);
           ptx::umma_commit_pair(&S.empty[s], 0x3);
           if (++s == kStages) {
             s = 0;
@@ -300,7 +324,7 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     const int bar_dec = 1 + 3 * xp, bar_free = 2 + 3 * xp, bar_full = 3 + 3 * xp;
     int nt = 0;
     for (int tile = pair; tile < total; tile += npairs, ++nt) {
-      const PairGeom G = pair_geom<MODE>(args, S, tile, R, rank, plane_rows);
+      const PairGeom G = pair_geom<MODE, KSUB>(args, S, tile, R, rank, plane_rows);
       const Tile& tl = G.t;
       const int slot = nt & 1;
       const uint32_t use = (uint32_t)(nt >> 1);
@@ -433,16 +457,16 @@ bool make_pair_maps(PairMaps* b, const void* base, uint64_t inner, uint64_t oute
   return true;
 }
 
-template <int MODE>
+template <int MODE, int KSUB>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& a_sh, const PairMaps& b,
                         const PairMaps& b_sh, const TcArgs& args, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int max_pairs = 0;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(tc2_grouped_kernel<MODE>,
+    attr_err = cudaFuncSetAttribute(tc2_grouped_kernel<MODE, KSUB>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)pair_smem_bytes());
+                                    (int)pair_smem_bytes<KSUB>());
     if (attr_err != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
@@ -452,10 +476,10 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& a_sh, const Pai
     at[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * (unsigned)sm_count(), 1, 1);
     cfg.blockDim = dim3(kThreads2, 1, 1);
-    cfg.dynamicSmemBytes = pair_smem_bytes();
+    cfg.dynamicSmemBytes = pair_smem_bytes<KSUB>();
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    attr_err = cudaOccupancyMaxActiveClusters(&max_pairs, tc2_grouped_kernel<MODE>, &cfg);
+    attr_err = cudaOccupancyMaxActiveClusters(&max_pairs, tc2_grouped_kernel<MODE, KSUB>, &cfg);
     if (attr_err == cudaSuccess && max_pairs < 1) attr_err = cudaErrorInvalidConfiguration;
   });
   if (attr_err != cudaSuccess) return attr_err;
@@ -467,11 +491,11 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& a_sh, const Pai
   at[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2 * (unsigned)max_pairs, 1, 1);
   cfg.blockDim = dim3(kThreads2, 1, 1);
-  cfg.dynamicSmemBytes = pair_smem_bytes();
+  cfg.dynamicSmemBytes = pair_smem_bytes<KSUB>();
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc2_grouped_kernel<MODE>, a, a_sh, b, b_sh, args);
+  return cudaLaunchKernelEx(&cfg, tc2_grouped_kernel<MODE, KSUB>, a, a_sh, b, b_sh, args);
 }
 
 }  // namespace
@@ -492,7 +516,7 @@ cudaError_t launch_tc2_gate_up(const moe_shape& s, const Layout& L, char* ws, co
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
   LaunchScope scope(MOE_K_GATE_UP, st);
-  return launch_pair<kPairGateUp>(a, a_sh, b, b_sh, args, st);
+  return launch_pair<kPairGateUp, 2>(a, a_sh, b, b_sh, args, st);
 }
 
 cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
@@ -513,7 +537,9 @@ cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
   args.y_shared = y_shared;
   args.out = out;
   LaunchScope scope(MOE_K_DOWN, st);
-  return launch_pair<kPairDown>(a, a_sh, b, b, args, st);
+  // 128-K stages for long down loops (I >= 1024); 64-K stages and a 6-deep ring otherwise
+  if (s.I >= 1024 && s.Is >= 1024) return launch_pair<kPairDown, 2>(a, a_sh, b, b, args, st);
+  return launch_pair<kPairDown, 1>(a, a_sh, b, b, args, st);
 }
 
 }  // namespace moe
