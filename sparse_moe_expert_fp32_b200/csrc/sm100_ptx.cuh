@@ -259,10 +259,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t cta_addr, uint32_t rank
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (this CTA's or the peer's),
-// releasing this thread's prior memory operations at cluster scope.
+// with the default semantics (release at CTA scope). A cluster-scope release would make the
+// arriving thread wait until its earlier global atomics had reached L2 ("membar" stalls in
+// the down epilogue); what the arrive must order (tensor-memory reads) is ordered by
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // 2-D tiled load into this CTA's shared memory whose completed bytes are counted on the
