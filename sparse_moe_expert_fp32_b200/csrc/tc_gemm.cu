@@ -260,7 +260,11 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     bool aborted = false;
     const int plane_rows = (MODE == kDown) ? (int)(args.h_plane / (size_t)args.ldh) : 0;
     // tiles are handed out in order by one counter: neighbouring tiles (the chunks of one
-    // weight tile, the M tiles of one expert) run at the same time on neighbouring SMs
+    // weight tile, the M tiles of one expert) run at the same time on neighbouring SMs.
+    // Lane 0 asks for the next tile one tile ahead, so the counter's round trip to L2 hides
+    // behind the current tile's copies instead of stalling them (short decode tiles paid
+    // it once per tile).
+    int ahead = (lane == 0) ? atomicAdd(args.counter, 1) : 0;
     for (int qi = 0; !aborted; ++qi) {
       const int slot = qi % kQueue;
       int tile = 0;
@@ -268,8 +272,9 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (!wait_phase(&S.q_empty[slot], ((uint32_t)(qi / kQueue) & 1u) ^ 1u, S, args.status)) {
           tile = -2;
         } else {
-          tile = atomicAdd(args.counter, 1);
+          tile = ahead;
           if (tile >= total) tile = -1;
+          else ahead = atomicAdd(args.counter, 1);
           S.q[slot] = tile;
           ptx::mbar_arrive(&S.q_full[slot]);
         }
