@@ -246,6 +246,31 @@ def dist_setup():
     return world, rank, local
 
 
+def dist_barrier(world: int) -> None:
+    """Barrier over the ranks of the job (no-op on one process)."""
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def dist_max(v: float, world: int, device) -> float:
+    """The largest of every rank's `v` (each rank's device time: the job takes the slowest)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(tokens_per_rank_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job throughput in tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank_step * steps * world / (ms / 1e3)
+
+
 def run_reference(args, cfg, world, rank):
     if rank != 0:
         return None
@@ -326,19 +351,10 @@ def run_ours(args, cfg, world, rank, local):
         time.sleep(1.5)  # nvidia-smi start-up
 
     def barrier():
-        if world > 1:
-            import torch.distributed as dist
-
-            dist.barrier()
+        dist_barrier(world)
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        import torch.distributed as dist
-
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return dist_max(v, world, "cuda")
 
     # ---- device-resident timed region: one layer forward per step, replayed from a CUDA
     # graph (as a served layer would run; --no-graph launches every kernel from the host)
@@ -412,8 +428,7 @@ def run_ours(args, cfg, world, rank, local):
     if rank != 0:
         return None
 
-    tokens = cfg.T * args.steps * world
-    value = tokens / (ms / 1e3)
+    value = job_value(cfg.T, args.steps, world, ms)
     peaks, peak_kind = load_peaks()
     kernels = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": None}
                for k, v in prof.items() if v[1] > 0}
@@ -445,7 +460,7 @@ def run_ours(args, cfg, world, rank, local):
             "zero_channel_compaction": compact,
             "roofline": roofline,
             "graph": not args.no_graph,
-            "e2e": {"value": cfg.T * args.steps * world / (ms_e2e / 1e3), "unit": "tokens/s",
+            "e2e": {"value": job_value(cfg.T, args.steps, world, ms_e2e), "unit": "tokens/s",
                     "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 4},
             "gpu_launches": launches, "kernels": kernels,
             "clocks": sampler.summary(windows) if sampler else None}
