@@ -275,6 +275,8 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       uint32_t ph = 0;
       bool aborted = false;
       const uint64_t desc0 = ptx::smem_desc_kmajor<kRowB>(smem);  // stage 0, A operand
+      // readiness of the next stage, tested while the current stage's MMAs are queued
+      bool ready = ptx::mbar_test_wait(&S.full[0], 0);
       for (int tile = pair; tile < total && !aborted; tile += npairs, ++nt) {
         const PairGeom G = pair_geom<MODE, KSUB>(args, S, tile, R, rank, plane_rows);
         const int slot = nt & 1;
@@ -289,19 +291,26 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         for (int ks = 0; ks < G.nk; ++ks) {
           // The copies' completion on the full barrier orders them before the MMAs that
           // read the stage; no tcgen05 fence is needed here.
-          if (!wait_phase(&S.full[s], ph, S, args.status)) {
+          if (!ready && !wait_phase(&S.full[s], ph, S, args.status)) {
             aborted = true;
             break;
           }
+          const int s2 = (s + 1 == kStages) ? 0 : s + 1;
+          const uint32_t ph2 = (s2 == 0) ? (ph ^ 1u) : ph;
           const uint64_t ad = desc0 + (uint64_t)s * (kStageBytes >> 4);
-          ptx::umma_bf16_pair_x4(d, ad, ad + (kABytes >> 4), idesc, ks > 0 ? 1u : 0u);
-          if (KSUB == 2)
-            ptx::umma_bf16_pair_x4(d, ad + (kASub >> 4), ad + ((kABytes + kBSub) >> 4), idesc, 1u);
-          ptx::umma_commit_pair(&S.empty[s], 0x3);
-          if (++s == kStages) {
-            s = 0;
-            ph ^= 1u;
+          const uint64_t bd = ad + (kABytes >> 4);
+          if (KSUB == 2) {
+            ptx::umma_bf16_pair_x4(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            ready = ptx::mbar_test_wait(&S.full[s2], ph2);
+            ptx::umma_bf16_pair_x4(d, ad + (kASub >> 4), bd + (kBSub >> 4), idesc, 1u);
+          } else {
+            ptx::umma_bf16_pair_x2(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            ready = ptx::mbar_test_wait(&S.full[s2], ph2);
+            ptx::umma_bf16_pair_x2(d, ad + 4, bd + 4, idesc, 1u);
           }
+          ptx::umma_commit_pair(&S.empty[s], 0x3);
+          s = s2;
+          ph = ph2;
         }
         if (aborted) break;
         ptx::umma_commit_pair(&S.tmem_full[slot], 0x3);

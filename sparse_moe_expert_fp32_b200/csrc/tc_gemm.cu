@@ -345,6 +345,8 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       bool aborted = false;
       const uint64_t desc0 = ptx::smem_desc_kmajor<C::kRowBytes>(smem);  // stage 0, first A tile
       constexpr uint64_t kDA = C::kATileBytes >> 4, kDB = C::kBTileBytes >> 4;
+      // readiness of the next stage, tested while the current stage's MMAs are queued
+      bool ready = ptx::mbar_test_wait(&S.full[0], 0);
       for (int qi = 0; !aborted; ++qi) {
         const int slot = qi % kQueue;
         if (!wait_phase(&S.q_full[slot], (uint32_t)(qi / kQueue) & 1u, S, args.status)) {
@@ -370,24 +372,25 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         for (int ks = 0; ks < G.nk; ++ks) {
           // The copies' completion on the full barrier orders them before the MMAs that
           // read the stage; no tcgen05 fence is needed here.
-          if (!wait_phase(&S.full[s], ph, S, args.status)) {
+          if (!ready && !wait_phase(&S.full[s], ph, S, args.status)) {
             aborted = true;
             break;
           }
+          const int s2 = (s + 1 == C::kStages) ? 0 : s + 1;
+          const uint32_t ph2 = (s2 == 0) ? (ph ^ 1u) : ph;
           const uint64_t a0 = desc0 + (uint64_t)s * (C::kStageBytes >> 4);
           const uint64_t bd = a0 + 2 * kDA;
           const uint32_t acc = ks > 0 ? 1u : 0u;
           ptx::umma_bf16_x4(d0, a0, bd, idesc, acc);
+          ready = ptx::mbar_test_wait(&S.full[s2], ph2);
           ptx::umma_bf16_x4(d1, a0 + kDA, bd, idesc, acc);
           if (MODE == kDown) {  // the lo half of h into the same accumulators
             ptx::umma_bf16_x4(d0, a0, bd + kDB, idesc, 1u);
             ptx::umma_bf16_x4(d1, a0 + kDA, bd + kDB, idesc, 1u);
           }
           ptx::umma_commit(&S.empty[s]);
-          if (++s == C::kStages) {
-            s = 0;
-            ph ^= 1u;
-          }
+          s = s2;
+          ph = ph2;
         }
         if (aborted) break;
         for (int i = 0; i < count; ++i) ptx::umma_commit(&S.tmem_full[(first + i) & 1]);
