@@ -73,9 +73,10 @@ typedef struct moe_weights {
 /* Grouped-GEMM variant used by moe_grouped_swiglu and moe_layer_forward. */
 typedef enum moe_variant {
   MOE_VARIANT_AUTO = 0,   /* tensor-core kernels where the shape allows (I, Is multiples of
-                             128, H of 256), else the streaming kernels: the CTA-pair
-                             kernels when the batch averages at least 16 routed rows per
-                             expert (T*k >= 16*E), else the one-CTA kernels               */
+                             128, H of 256), else the streaming kernels: the down GEMM on
+                             CTA pairs; the gate|up GEMM on CTA pairs when the batch
+                             averages at least 16 routed rows per expert (T*k >= 16*E),
+                             else one CTA per tile                                        */
   MOE_VARIANT_STREAM = 1, /* weight-streaming CUDA-core kernels                             */
   MOE_VARIANT_TC = 2,     /* tcgen05/TMEM grouped GEMMs fed by TMA, one CTA per tile (falls
                              back to streaming for shapes they do not support)             */

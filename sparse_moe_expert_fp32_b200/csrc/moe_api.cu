@@ -150,14 +150,20 @@ bool use_tc(const moe_shape& s) {
   return tc_supported(s);
 }
 
-// CTA-pair kernels for this shape? They pay off once the token tiles are wide: AUTO takes
-// them when the batch averages at least 16 routed rows per expert (B200: 2.4T-shaped
-// prefill gate|up 6.92 ms against 6.99, down 6.94 against 8.00; Flash-Next-shaped prefill
-// gate|up 0.71 against 0.78; at decode sizes the one-CTA kernels' 16-token tiles suffice).
-bool use_tc2(const moe_shape& s) {
+// CTA-pair kernels for this shape, per GEMM? Measured on B200 (µs per launch, one-CTA /
+// pair): the down GEMM is faster on pairs at every size (Flash-Next decode 234 / 220,
+// 2.4T-shaped prefill 8001 / 6941); the gate|up GEMM only once the token tiles are wide
+// (decode 384 / 393; 2.4T-shaped prefill 6986 / 6921; Flash-Next prefill 780 / 709), which
+// AUTO takes as an average of at least 16 routed rows per expert.
+bool use_tc2_gate_up(const moe_shape& s) {
   const int v = g_variant.load();
   if (v == MOE_VARIANT_TC2) return true;
   return v == MOE_VARIANT_AUTO && (int64_t)s.T * s.k >= 16 * (int64_t)s.E;
+}
+
+bool use_tc2_down(const moe_shape& s) {
+  const int v = g_variant.load();
+  return v == MOE_VARIANT_TC2 || v == MOE_VARIANT_AUTO;
 }
 
 // Stage 4 on the plan in the workspace: fused (out != NULL) or per-row y / y_shared.
@@ -166,13 +172,12 @@ moe_status run_grouped(const moe_shape& s, const Layout& L, char* ws, const uint
                        const moe_weights& w, float* y, float* y_shared, float* out,
                        cudaStream_t st) {
   if (use_tc(s)) {
-    if (use_tc2(s)) {
-      MOE_CUDA(launch_tc2_gate_up(s, L, ws, x, sorted_token, w, st));
+    if (use_tc2_gate_up(s)) MOE_CUDA(launch_tc2_gate_up(s, L, ws, x, sorted_token, w, st));
+    else MOE_CUDA(launch_tc_gate_up(s, L, ws, x, sorted_token, w, st));
+    if (use_tc2_down(s))
       MOE_CUDA(launch_tc2_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));
-    } else {
-      MOE_CUDA(launch_tc_gate_up(s, L, ws, x, sorted_token, w, st));
+    else
       MOE_CUDA(launch_tc_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));
-    }
   } else {
     MOE_CUDA(launch_stream_gate_up(s, L, ws, x, sorted_token, w, st));
     MOE_CUDA(launch_stream_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));

@@ -19,6 +19,8 @@ import synth  # noqa: E402
 from parity_util import NEAR_TIE_GAP, assert_layer_close, err_stats, id_sets_match  # noqa: E402
 
 VARIANTS = {"stream": moe.MOE_VARIANT_STREAM, "tc": moe.MOE_VARIANT_TC, "tc2": moe.MOE_VARIANT_TC2}
+# AUTO mixes them by shape (at decode sizes: one-CTA gate|up, CTA-pair down)
+VARIANTS_AUTO = dict(VARIANTS, auto=moe.MOE_VARIANT_AUTO)
 
 
 def _u16(t):
@@ -257,13 +259,13 @@ def test_combine_exact_inputs():
 # ----------------------------------------------------------------------------- whole layer
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("variant", sorted(VARIANTS))
+@pytest.mark.parametrize("variant", sorted(VARIANTS_AUTO))
 @pytest.mark.parametrize("name", ["tiny", "flash_decode"])
 def test_layer_forward_full(name, variant):
     cfg = synth.CONFIGS[name]
     dev = synth.device_inputs(cfg, seed=0)
     host = synth.host_inputs(cfg, seed=0)
-    out, ids, _, _ = _forward(cfg, dev, VARIANTS[variant])
+    out, ids, _, _ = _forward(cfg, dev, VARIANTS_AUTO[variant])
     stats, ties = _check_layer(cfg, host, out, ids, list(range(cfg.T)))
     print(name, variant, stats, "near-ties", ties)
 
@@ -298,13 +300,13 @@ EDGE = {
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("variant", sorted(VARIANTS))
+@pytest.mark.parametrize("variant", sorted(VARIANTS_AUTO))
 @pytest.mark.parametrize("case", sorted(EDGE))
 def test_layer_edge_cases(case, variant):
     cfg = synth.CONFIGS["tiny"].replace(name=case, **EDGE[case])
     dev = synth.device_inputs(cfg, seed=5)
     host = synth.host_inputs(cfg, seed=5)
-    out, ids, tw, _ = _forward(cfg, dev, VARIANTS[variant])
+    out, ids, tw, _ = _forward(cfg, dev, VARIANTS_AUTO[variant])
     _check_layer(cfg, host, out, ids, list(range(cfg.T)))
     if cfg.k == 1:
         assert (tw == 1.0).all()
