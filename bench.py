@@ -169,11 +169,16 @@ def stored_traffic(kernel: str, workload: str):
 
 
 def source_hash(kernel: str) -> str:
+    """Hash of the code (comments and whitespace removed) of the files a kernel is built from:
+    a stored ncu traffic figure stays valid across comment edits, not across code changes."""
     hsh = hashlib.sha256()
     for f in KERNEL_SOURCES.get(kernel, ()):
         p = os.path.join(ROOT, "sparse_moe_expert_fp32_b200", "csrc", f)
         if os.path.exists(p):
-            hsh.update(open(p, "rb").read())
+            src = open(p, encoding="utf-8").read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            src = re.sub(r"//[^\n]*", "", src)
+            hsh.update(re.sub(r"\s+", "", src).encode())
     return hsh.hexdigest()
 
 
