@@ -74,6 +74,14 @@ __host__ __device__ inline PlanView plan_view(void* base, int E) {
 // Tensor-core tiling of a group with n rows into ceil(n / max) token chunks of nearly equal
 // size (multiples of 16 rows): max 256 rows for the gate|up GEMM, 128 for the down GEMM.
 constexpr int kTcChunkDown = 128;
+// Rows per gate|up tile: decode-size batches (T*k < 16*E, a few rows per expert) chunk at
+// kTcChunkSmall, so that the one-CTA gate|up kernel's stages can be small and more of them
+// fit; larger batches at kTcChunk. The plan builder and both gate|up kernels call this with
+// the same T, k, E.
+constexpr int kTcChunkSmall = 64;
+__host__ __device__ inline int tc_gate_up_chunk(int T, int k, int E) {
+  return (long long)T * k < 16LL * E ? kTcChunkSmall : kTcChunk;
+}
 __host__ __device__ inline int tc_nchunks(int n, int max_rows) {
   return (n + max_rows - 1) / max_rows;
 }

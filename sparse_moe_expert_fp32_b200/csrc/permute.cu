@@ -87,7 +87,7 @@ __device__ int block_exclusive_scan(int v, int* smem_warp, int* total) {
 
 // Group sizes n_g (g < E routed, g == E shared = T) -> plan. Called by all threads of a
 // kScanThreads CTA; thread g handles group g (E + 1 <= 1025: thread 0 also takes E).
-__device__ void build_plan(const int* n_of, int E, int H, int I, int Is,
+__device__ void build_plan(const int* n_of, int E, int H, int I, int Is, int T, int k,
                            PlanView pv, int* smem) {
   // thread g takes group g (g <= E); with E == 1024 the last thread also takes group E
   const int g = threadIdx.x;
@@ -103,7 +103,8 @@ __device__ void build_plan(const int* n_of, int E, int H, int I, int Is,
   if (threadIdx.x == 0) *pv.n_active = tot;
 
   auto inter = [&](int grp) { return grp < E ? I : Is; };
-  const int c0 = tc_nchunks(n0, kTcChunk), c1 = tc_nchunks(n1, kTcChunk);
+  const int uc = tc_gate_up_chunk(T, k, E);
+  const int c0 = tc_nchunks(n0, uc), c1 = tc_nchunks(n1, uc);
   const int d0 = tc_nchunks(n0, kTcChunkDown), d1 = tc_nchunks(n1, kTcChunkDown);
   const int t1a = (g <= E) ? c0 * (inter(g) / 128) : 0;
   const int t1b = has1 ? c1 * (Is / 128) : 0;
@@ -158,7 +159,7 @@ dispatch_scan_kernel(const int32_t* blk_count, int nblk, int T, int E, int k, in
     n_of[E] = T;
   }
   __syncthreads();
-  build_plan(n_of, E, H, I, Is, plan_view(plan_base, E), smem);
+  build_plan(n_of, E, H, I, Is, T, k, plan_view(plan_base, E), smem);
 }
 
 __global__ void __launch_bounds__(kPermBlock)
@@ -231,7 +232,7 @@ dispatch_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__
     n_of[E] = T;
   }
   __syncthreads();
-  build_plan(n_of, E, H, I, Is, plan_view(plan_base, E), smem);
+  build_plan(n_of, E, H, I, Is, T, k, plan_view(plan_base, E), smem);
   if (i < T) {
     const int word = i >> 5;
     const uint32_t below = (1u << (i & 31)) - 1u;
@@ -271,7 +272,7 @@ plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int T, int E, int 
     if (threadIdx.x == 0) set_flag(status, kFlagBounds);
   }
   __syncthreads();
-  build_plan(n_of, E, H, I, Is, plan_view(plan_base, E), smem);
+  build_plan(n_of, E, H, I, Is, T, k, plan_view(plan_base, E), smem);
 }
 
 }  // namespace

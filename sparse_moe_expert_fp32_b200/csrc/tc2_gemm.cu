@@ -130,7 +130,8 @@ __device__ __forceinline__ PairGeom pair_geom(const TcArgs& a, const PairShared&
                                               int R, int rank, int plane_rows) {
   constexpr int kStageK = Ring<KSUB>::kStageK;
   PairGeom G;
-  G.t = decode_tile(S.row0, S.tp, a.E, tile, MODE == kPairGateUp ? 256 : 128);
+  G.t = decode_tile(S.row0, S.tp, a.E, tile,
+                    MODE == kPairGateUp ? tc_gate_up_chunk(a.T, a.k, a.E) : kTcChunkDown);
   G.shared = G.t.g == a.E;
   if (MODE == kPairGateUp) {
     const int Ig = G.shared ? a.Is : a.I;

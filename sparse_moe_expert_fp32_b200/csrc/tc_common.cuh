@@ -20,7 +20,7 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;  // waits while leaving after a
 
 struct TcArgs {
   const int* plan;
-  int E, H, I, Is, T, ldh;
+  int E, H, I, Is, T, k, ldh;
   size_t h_plane;
   const int32_t* sorted_token;
   const float* sorted_w;
@@ -160,6 +160,7 @@ TcArgs base_args(const moe_shape& s, const Layout& L, char* ws) {
   a.I = s.I;
   a.Is = s.Is;
   a.T = s.T;
+  a.k = s.k;
   a.ldh = L.ldh;
   a.h_plane = L.h_plane;
   a.h = reinterpret_cast<uint16_t*>(ws + L.h);

@@ -52,7 +52,13 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256;
 constexpr int kQueue = 4;  // tile ids handed from the producer to the MMA and epilogue roles
 
-enum Mode { kGateUp = 0, kDown = 1, kRouter = 2 };
+// kGateUpSmall: the gate|up GEMM for decode-size batches (T*k < 16*E), whose tiles are
+// chunked at 64 token rows: its stages reserve room for 64 rows instead of 256, so five of
+// them fit and about 170 KB of weights are in flight per SM instead of about 100 KB.
+enum Mode { kGateUp = 0, kDown = 1, kRouter = 2, kGateUpSmall = 3 };
+__host__ __device__ constexpr bool is_gate_up(int mode) {
+  return mode == kGateUp || mode == kGateUpSmall;
+}
 
 // Per-mode pipeline geometry. The down GEMM keeps tiles of at most 128 tokens: its K loop
 // is short (K = I), so its epilogue must overlap the next tile's MMAs (one TMEM slot per
@@ -61,18 +67,19 @@ template <int MODE>
 struct Cfg {
   static constexpr int kBK = 64;                                  // K per stage
   static constexpr int kRowBytes = kBK * 2;                       // 128 (= swizzle)
-  static constexpr int kMaxTile = (MODE == kGateUp) ? 256 : 128;  // tokens per tile
+  static constexpr int kMaxTile =  // tokens per tile
+      MODE == kGateUp ? kTcChunk : (MODE == kGateUpSmall ? kTcChunkSmall : 128);
   static constexpr uint32_t kATileBytes = 128u * kRowBytes;
   static constexpr uint32_t kBTileBytes = (uint32_t)kMaxTile * kRowBytes;
   static constexpr int kBTiles = (MODE == kDown) ? 2 : 1;  // down: hi and lo rows of h
   static constexpr uint32_t kStageBytes = 2 * kATileBytes + kBTiles * kBTileBytes;
-  static constexpr int kStages = 3;
+  static constexpr int kStages = MODE == kGateUpSmall ? 5 : 3;
   static constexpr int kKK = kBK / 16;  // MMAs (K = 16) per stage and accumulator
 };
 
 struct SharedState {
-  uint64_t full[4];
-  uint64_t empty[4];
+  uint64_t full[5];
+  uint64_t empty[5];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t q_full[kQueue];
@@ -91,7 +98,7 @@ constexpr size_t smem_bytes() {
   return 1024 + (size_t)Cfg<MODE>::kStages * Cfg<MODE>::kStageBytes + sizeof(SharedState);
 }
 static_assert(smem_bytes<kGateUp>() <= 232448 && smem_bytes<kDown>() <= 232448 &&
-                  smem_bytes<kRouter>() <= 232448,
+                  smem_bytes<kRouter>() <= 232448 && smem_bytes<kGateUpSmall>() <= 232448,
               "over the 227 KB of shared memory a CTA may use");
 
 // The token operand's tensor map in each box height (index i: 128 >> i rows).
@@ -156,7 +163,7 @@ __device__ __forceinline__ Geom tile_geom(const TcArgs& a, const SharedState& S,
   }
   G.t = decode_tile(S.row0, S.tp, a.E, tile, C::kMaxTile);
   G.shared = G.t.g == a.E;
-  if (MODE == kGateUp) {
+  if (is_gate_up(MODE)) {
     const int Ig = G.shared ? a.Is : a.I;
     const int base = G.shared ? 0 : G.t.g * 2 * a.I;
     G.a_row0 = base + G.t.m * 128;
@@ -206,7 +213,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   } else {
     // the plan is read on every tile by every role: keep it in shared memory
     const PlanView pv = plan_view(const_cast<int*>(args.plan), E);
-    const int* tp = (MODE == kGateUp) ? pv.tp1 : pv.tp2;
+    const int* tp = (is_gate_up(MODE)) ? pv.tp1 : pv.tp2;
     for (int g = threadIdx.x; g < E + 2; g += blockDim.x) {
       S.tp[g] = tp[g];
       S.row0[g] = pv.row0[g];
@@ -215,7 +222,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     R = pv.row0[E];
   }
 
-  if (MODE == kGateUp && blockIdx.x == 0 && threadIdx.x == 0) *args.counter_next = 0;
+  if (is_gate_up(MODE) && blockIdx.x == 0 && threadIdx.x == 0) *args.counter_next = 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       ptx::mbar_init(&S.full[s], 1);
@@ -298,7 +305,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (j < np * C::kBTiles) {
           const int plane = j / np;
           token_piece(G.t.N, j - plane * np, r, h);
-          const BMaps& bm = (MODE == kGateUp && G.shared) ? tm_b_sh : tm_b;
+          const BMaps& bm = (is_gate_up(MODE) && G.shared) ? tm_b_sh : tm_b;
           my_map = &bm.m[h];
           my_off = 2 * C::kATileBytes + plane * C::kBTileBytes + (uint32_t)r * C::kRowBytes;
           my_row = G.b_row0 + r + plane * plane_rows;
@@ -455,7 +462,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         ptx::tmem_ld32(b0 + c0, r0);
         ptx::tmem_ld32(b1 + c0, r1);
         ptx::tmem_ld_wait();
-        if (MODE == kGateUp) {
+        if (is_gate_up(MODE)) {
           const int ch = tl.m * 128 + qd * 32 + lane;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -658,7 +665,7 @@ cudaError_t launch_gather_rows(const moe_shape& s, const Layout& L, char* ws, co
 
 cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                               const int32_t* sorted_token, const moe_weights& w, cudaStream_t st) {
-  using C = Cfg<kGateUp>;
+  using C = Cfg<kGateUp>;  // kBK and box shapes are the same for kGateUpSmall
   uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
   {
     cudaError_t e = launch_gather_rows(s, L, ws, x, sorted_token, st);
@@ -676,6 +683,8 @@ cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, con
   args.counter = reinterpret_cast<int*>(ws + L.sched) + 0;
   args.counter_next = reinterpret_cast<int*>(ws + L.sched) + 1;
   LaunchScope scope(MOE_K_GATE_UP, st);
+  if (tc_gate_up_chunk(s.T, s.k, s.E) == kTcChunkSmall)
+    return launch_mode<kGateUpSmall>(a, a_sh, b, b_sh, args, sm_count(), st);
   return launch_mode<kGateUp>(a, a_sh, b, b_sh, args, sm_count(), st);
 }
 
