@@ -550,8 +550,12 @@ cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
   args.y_shared = y_shared;
   args.out = out;
   LaunchScope scope(MOE_K_DOWN, st);
-  // 128-K stages for long down loops (I >= 1024); 64-K stages and a 6-deep ring otherwise
-  if (s.I >= 1024 && s.Is >= 1024) return launch_pair<kPairDown, 2>(a, a_sh, b, b, args, st);
+  // 128-K stages (eight MMAs per producer/issuer hand-off) for long down loops (I >= 1024)
+  // and for decode-size batches, whose tiny MMAs (N = 2 x a few rows) leave the issuing
+  // thread as the bound with the copies landing far ahead; 64-K stages and a 6-deep ring
+  // for short loops at prefill sizes (inter 640: 5 stages per tile)
+  if ((s.I >= 1024 && s.Is >= 1024) || (int64_t)s.T * s.k < 16 * (int64_t)s.E)
+    return launch_pair<kPairDown, 2>(a, a_sh, b, b, args, st);
   return launch_pair<kPairDown, 1>(a, a_sh, b, b, args, st);
 }
 
