@@ -329,6 +329,24 @@ def test_hot_expert_many_tokens(variant):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("variant", sorted(VARIANTS_AUTO))
+def test_hot_expert_decode_geometry(variant):
+    """Decode-size shape (T*k < 16*E: 64-row gate|up tiles) with every token on expert 7:
+    200 rows in one group and 200 shared rows, so both split into several 64-row tiles."""
+    cfg = synth.CONFIGS["tiny"].replace(name="hot_decode", T=200, E=256, k=4)
+    assert cfg.T * cfg.k < 16 * cfg.E
+    dev = synth.device_inputs(cfg, seed=8)
+    bias = np.zeros(cfg.E, np.float32)
+    bias[7] = 50.0
+    dev["router_bias"] = _dev_f32(bias)
+    host = synth.host_inputs(cfg, seed=8)
+    host.router_bias = bias
+    out, ids, _, _ = _forward(cfg, dev, VARIANTS_AUTO[variant])
+    assert (ids == 7).any(axis=1).all()
+    _check_layer(cfg, host, out, ids, list(range(cfg.T)))
+
+
+@pytest.mark.gpu
 def test_empty_batch_and_host_entry():
     cfg = synth.CONFIGS["tiny"]
     dev = synth.device_inputs(cfg, seed=0)
