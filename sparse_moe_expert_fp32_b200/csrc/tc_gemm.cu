@@ -13,10 +13,12 @@
 //     token rows, copied beforehand in dispatch order (gather_rows_kernel) so that a token
 //     tile is a few plain 2-D TMA boxes. Epilogue: h = SiLU(gate) * up stored as the bf16
 //     pair hi = bf16(h), lo = bf16(h - hi).
-//   down: 256 rows of one expert's W_down against its packed rows; per K step two MMAs add
-//     W h_hi and W h_lo into the same accumulators. Epilogue: y rows (staged path) or
-//     routing-weight-scaled fp32 atomic adds into out[token] ("Weighted combine + gated
-//     shared expert").
+//   down: 256 rows of one expert's W_down against its packed rows. The tile's h_lo rows
+//     follow its h_hi rows in shared memory, so one MMA per accumulator with N = 2 x rows
+//     yields W h_hi in columns [0, N) and W h_lo in [N, 2N), added in the epilogue (half
+//     the MMA instructions of two N-wide MMAs; at decode sizes the issuing thread is the
+//     bound). Epilogue: y rows (staged path) or routing-weight-scaled fp32 atomic adds
+//     into out[token] ("Weighted combine + gated shared expert").
 //   router: 256 experts x 128 tokens of logits = x . (hi + mid + lo)^T, K = 3H over the
 //     exact bf16 split of the fp32 router matrix.
 //
@@ -185,8 +187,10 @@ __device__ __forceinline__ Geom tile_geom(const TcArgs& a, const SharedState& S,
 struct Slots {
   int next = 0;
   uint32_t uses[2] = {0u, 0u};
-  __device__ __forceinline__ void take(int N, int& first, int& count) const {
-    count = N > 128 ? 2 : 1;
+  // cols: TMEM columns one accumulator of the tile needs (N; 2N for the down GEMM, whose
+  // hi and lo halves of h share one MMA)
+  __device__ __forceinline__ void take(int cols, int& first, int& count) const {
+    count = cols > 128 ? 2 : 1;
     first = count == 2 ? 0 : next;
   }
   __device__ __forceinline__ void done(int first, int count) {
@@ -307,7 +311,8 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           token_piece(G.t.N, j - plane * np, r, h);
           const BMaps& bm = (is_gate_up(MODE) && G.shared) ? tm_b_sh : tm_b;
           my_map = &bm.m[h];
-          my_off = 2 * C::kATileBytes + plane * C::kBTileBytes + (uint32_t)r * C::kRowBytes;
+          // down: the lo rows follow the hi rows, so one MMA with N = 2 x rows reads both
+          my_off = 2 * C::kATileBytes + (uint32_t)(plane * G.t.N + r) * C::kRowBytes;
           my_row = G.b_row0 + r + plane * plane_rows;
         }
       }
@@ -351,7 +356,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       Slots sl;
       bool aborted = false;
       const uint64_t desc0 = ptx::smem_desc_kmajor<C::kRowBytes>(smem);  // stage 0, first A tile
-      constexpr uint64_t kDA = C::kATileBytes >> 4, kDB = C::kBTileBytes >> 4;
+      constexpr uint64_t kDA = C::kATileBytes >> 4;
       // readiness of the next stage, tested while the current stage's MMAs are queued
       bool ready = ptx::mbar_test_wait(&S.full[0], 0);
       for (int qi = 0; !aborted; ++qi) {
@@ -364,9 +369,10 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         ptx::mbar_arrive(&S.q_empty[slot]);
         if (tile < 0) break;
         const Geom G = tile_geom<MODE>(args, S, tile, R);
-        const uint32_t idesc = ptx::idesc_bf16_f32(128, G.t.N);
+        const int cols = MODE == kDown ? 2 * G.t.N : G.t.N;  // down: columns [0,N) hi, [N,2N) lo
+        const uint32_t idesc = ptx::idesc_bf16_f32(128, cols);
         int first, count;
-        sl.take(G.t.N, first, count);
+        sl.take(cols, first, count);
         for (int i = 0; i < count && !aborted; ++i) {
           const int sidx = (first + i) & 1;
           if (!wait_phase(&S.tmem_empty[sidx], (sl.uses[sidx] & 1u) ^ 1u, S, args.status))
@@ -391,10 +397,6 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           ptx::umma_bf16_x4(d0, a0, bd, idesc, acc);
           ready = ptx::mbar_test_wait(&S.full[s2], ph2);
           ptx::umma_bf16_x4(d1, a0 + kDA, bd, idesc, acc);
-          if (MODE == kDown) {  // the lo half of h into the same accumulators
-            ptx::umma_bf16_x4(d0, a0, bd + kDB, idesc, 1u);
-            ptx::umma_bf16_x4(d1, a0 + kDA, bd + kDB, idesc, 1u);
-          }
           ptx::umma_commit(&S.empty[s]);
           s = s2;
           ph = ph2;
@@ -427,7 +429,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       const Geom G = tile_geom<MODE>(args, S, tile, R);
       const Tile& tl = G.t;
       int first, count;
-      sl.take(tl.N, first, count);
+      sl.take(MODE == kDown ? 2 * tl.N : tl.N, first, count);
       const uint32_t b0 = tmem + lane_off + first * kSlotCols;
       const uint32_t b1 = b0 + (count == 2 ? kSlotCols : 128u);
       // down: token and weight of this warp's columns, requested before waiting for the
@@ -461,7 +463,21 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         uint32_t r0[32], r1[32];
         ptx::tmem_ld32(b0 + c0, r0);
         ptx::tmem_ld32(b1 + c0, r1);
-        ptx::tmem_ld_wait();
+        if (MODE == kDown) {
+          // add the lo half (columns N + c0 ..; they stay inside this accumulator's region:
+          // c0 < N, so N + c0 + 31 < 128 for N <= 64 and < 256 for N <= 128)
+          uint32_t l0[32], l1[32];
+          ptx::tmem_ld32(b0 + tl.N + c0, l0);
+          ptx::tmem_ld32(b1 + tl.N + c0, l1);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            r0[j] = __float_as_uint(__uint_as_float(r0[j]) + __uint_as_float(l0[j]));
+            r1[j] = __float_as_uint(__uint_as_float(r1[j]) + __uint_as_float(l1[j]));
+          }
+        } else {
+          ptx::tmem_ld_wait();
+        }
         if (is_gate_up(MODE)) {
           const int ch = tl.m * 128 + qd * 32 + lane;
 #pragma unroll
