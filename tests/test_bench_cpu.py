@@ -1,0 +1,60 @@
+"""CPU checks of bench.py's arithmetic: the algorithmic bytes and FLOPs behind the roofline
+fraction, the job-wide value, and the source hash that ties a stored ncu traffic figure to
+the kernel code."""
+import os
+import shutil
+
+import pytest
+
+import bench
+import synth
+
+
+def test_decode_gate_up_bytes_by_hand():
+    # Flash-Next decode, 370 activated experts: each holds gate and up rows [2*640][2560]
+    # in bf16; plus the shared expert's, the 64 token rows, and h as a bf16 hi/lo pair for
+    # the 640 routed rows and the 64 shared rows.
+    cfg = synth.CONFIGS["flash_decode"]
+    weights = (370 * 2 * 640 * 2560 + 2 * 640 * 2560) * 2
+    x = 64 * 2560 * 2
+    h = (640 * 640 + 64 * 640) * 2 * 2
+    assert bench.algorithmic_bytes("gate_up", cfg, 370) == weights + x + h == 2433515520
+
+
+def test_decode_down_bytes_by_hand():
+    cfg = synth.CONFIGS["flash_decode"]
+    weights = (370 * 2560 * 640 + 2560 * 640) * 2
+    h = (640 * 640 + 64 * 640) * 2 * 2
+    out = 64 * 2560 * 4
+    assert bench.algorithmic_bytes("down", cfg, 370) == weights + h + out == 1218150400
+
+
+def test_prefill_flops_match_the_layer_count():
+    # 6*H*I per routed assignment plus 6*H*Is per token for the shared expert, split 2:1
+    # between gate|up and down (the survey's 805.3 G + 80.5 G for the Flash-Next prefill)
+    cfg = synth.CONFIGS["flash_prefill"]
+    total = bench.kernel_flops("gate_up", cfg) + bench.kernel_flops("down", cfg)
+    assert total == 6 * (cfg.R * cfg.H * cfg.I + cfg.T * cfg.H * cfg.Is)
+    assert total == pytest.approx(805.3e9 + 80.5e9, rel=1e-3)
+    assert bench.kernel_flops("gate_up", cfg) == 2 * bench.kernel_flops("down", cfg)
+
+
+def test_job_value_counts_every_rank():
+    assert bench.job_value(64, 200, 1, 120.0) == pytest.approx(64 * 200 / 0.12)
+    assert bench.job_value(64, 200, 8, 120.0) == pytest.approx(8 * 64 * 200 / 0.12)
+
+
+def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+    csrc = tmp_path / "sparse_moe_expert_fp32_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    real = os.path.join(bench.ROOT, "sparse_moe_expert_fp32_b200", "csrc")
+    for f in bench.KERNEL_SOURCES["down"]:
+        shutil.copy(os.path.join(real, f), csrc / f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.source_hash("down")
+    p = csrc / "tc2_gemm.cu"
+    src = p.read_text()
+    p.write_text("// a new comment line\n" + src.replace("\n", "\n  ", 3) + "\n/* and a block */\n")
+    assert bench.source_hash("down") == h0
+    p.write_text(src.replace("kSlotCols = 256", "kSlotCols = 255", 1))
+    assert bench.source_hash("down") != h0
