@@ -114,17 +114,24 @@ def shared_gate(x_bf16: np.ndarray, w_shared_gate: np.ndarray) -> np.ndarray:
 def swiglu_expert(x64: np.ndarray, w_gate_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
     """W_down (SiLU(W_gate x) * W_up x) for each row of x64 [n][H].
 
-    w_gate_up: uint16 [2I][H] (rows 0..I-1 gate, I..2I-1 up); w_down: uint16 [H][I].
+    w_gate_up: [2I][H] (rows 0..I-1 gate, I..2I-1 up); w_down: [H][I]; each as bf16 bit
+    patterns (uint16) or fp64 values.
     """
     H = x64.shape[1]
     two_i, hh = w_gate_up.shape
     I = two_i // 2
     assert hh == H and w_down.shape == (H, I), "expert weight shapes"
-    wgu = bf16_to_f64(w_gate_up)
+    wgu = _weights_f64(w_gate_up)
     g = x64 @ wgu[:I].T
     u = x64 @ wgu[I:].T
     h = silu(g) * u
-    return h @ bf16_to_f64(w_down).T
+    return h @ _weights_f64(w_down).T
+
+
+def _weights_f64(w: np.ndarray) -> np.ndarray:
+    """Weights as fp64: uint16 arrays are bf16 bit patterns; float64 arrays are values
+    already (the dequantised FP8 experts)."""
+    return w if w.dtype == np.float64 else bf16_to_f64(w)
 
 
 def _expert(bank: ArrayOrFn, e: int) -> np.ndarray:
@@ -165,6 +172,104 @@ def compact_zero_channels(w_gate_up: np.ndarray, w_down: np.ndarray, I_c: int):
         gu[e, I_c:I_c + n] = w_gate_up[e, I + keep]
         dn[e, :, :n] = w_down[e][:, keep]
     return gu, dn
+
+
+# --------------------------------------------------------------------------- FP8 experts
+# Source: "Qwen3.8, weights in hand: 98% of a 2.4T model is routed experts", section "What
+# FP8 actually quantizes": the FP8 checkpoint stores the routed experts at one byte per
+# parameter and keeps the router, the shared expert and its gate in bf16. The page names
+# neither the 8-bit format nor the scaling. Reading taken here: E4M3 codes (1 sign bit,
+# 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest finite value 448,
+# 0x7F / 0xFF reserved for NaN) with one fp32 scale per weight row (a row of W_gate|up is
+# one output channel over H, a row of W_down one output channel over I):
+#   scale = fp32(amax_row / 448)        (amax of the bf16 row; scale = 0 for a zero row)
+#   code  = E4M3 round-to-nearest-even of fp32(w / scale), clamped to +-448
+# Both divisions are IEEE fp32 divisions; the dequantised weight is decode(code) * scale,
+# exact in fp64. Activations stay bf16.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """uint8 E4M3 codes -> fp64 values, from the format's definition (NaN codes -> nan)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    normal = np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64))
+    sub = m * 2.0 ** -9
+    v = np.where(e == 0, sub, normal)
+    v = np.where((c & 0x7F) == 0x7F, np.nan, v)
+    return sign * v
+
+
+def e4m3_encode(q: np.ndarray) -> np.ndarray:
+    """fp32 values -> uint8 E4M3 codes: nearest representable value, ties to the even
+    mantissa, magnitudes above 448 clamped to 448 (saturating, never NaN). Input must be
+    finite."""
+    a64 = np.abs(np.asarray(q, dtype=np.float32).astype(np.float64))
+    neg = np.signbit(np.asarray(q, dtype=np.float32))
+    code = np.zeros(a64.shape, dtype=np.int64)
+    # subnormal binade and below: multiples of 2^-9 (n = 8 is 2^-6, the first normal code)
+    small = a64 < 2.0 ** -6
+    code[small] = np.rint(a64[small] * 2.0 ** 9).astype(np.int64)
+    big = ~small
+    if big.any():
+        _, ex = np.frexp(a64[big])  # a = f * 2^ex, f in [0.5, 1)
+        e = ex - 1  # a in [2^e, 2^(e+1))
+        n = np.rint(np.ldexp(a64[big], (3 - e).astype(np.int64))).astype(np.int64)  # 8..16
+        carry = n == 16
+        e = np.where(carry, e + 1, e)
+        n = np.where(carry, 8, n)
+        code[big] = ((e + 7) << 3) | (n - 8)
+    code = np.minimum(code, 0x7E)  # 448
+    return (code | np.where(neg, 0x80, 0)).astype(np.uint8)
+
+
+def quantize_fp8_rows(w_bf16: np.ndarray):
+    """uint16 bf16 [rows][n] -> (uint8 E4M3 codes [rows][n], fp32 scales [rows]).
+
+    Every step in fp32 as stated above: amax of the row (exact), scale = amax / 448,
+    q = w / scale, code = e4m3_encode(q); a zero row gets scale 0 and code 0 everywhere.
+    """
+    w32 = bf16_to_f64(w_bf16).astype(np.float32)
+    amax = np.abs(w32).max(axis=-1)
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = (w32 / safe[..., None]).astype(np.float32)
+    codes = e4m3_encode(q)
+    codes[scale == 0] = 0
+    return codes, scale
+
+
+def dequantize_fp8_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """decode(code) * scale per row, fp64 (exact: a 4-bit significand times an fp32)."""
+    return e4m3_decode(codes) * np.asarray(scales, dtype=np.float32).astype(np.float64)[..., None]
+
+
+class Fp8Experts:
+    """The routed experts of a layer in FP8: quantised lazily per expert from the bf16
+    source bank (callables e -> uint16 slice) and returned dequantised (fp64), ready for
+    ``moe_forward``. ``codes_gate_up(e)`` etc. give the stored codes and scales."""
+
+    def __init__(self, gate_up: Callable[[int], np.ndarray], down: Callable[[int], np.ndarray]):
+        self._gu, self._dn = gate_up, down
+        self._cache: dict = {}
+
+    def quantized(self, e: int):
+        if e not in self._cache:
+            if len(self._cache) > 64:
+                self._cache.clear()
+            self._cache[e] = (quantize_fp8_rows(self._gu(e)), quantize_fp8_rows(self._dn(e)))
+        return self._cache[e]
+
+    def gate_up(self, e: int) -> np.ndarray:
+        (c, s), _ = self.quantized(e)
+        return dequantize_fp8_rows(c, s)
+
+    def down(self, e: int) -> np.ndarray:
+        _, (c, s) = self.quantized(e)
+        return dequantize_fp8_rows(c, s)
 
 
 # --------------------------------------------------------------------------- dispatch
@@ -254,9 +359,11 @@ def combine(y: np.ndarray, y_shared: np.ndarray, assign_row: np.ndarray, weights
     return out
 
 
-def forward_inputs(inp, rows=None, forced_ids=None) -> dict:
-    """moe_forward on a ``synth.HostInputs``; ``rows`` selects a token subset."""
+def forward_inputs(inp, rows=None, forced_ids=None, fp8: Optional[Fp8Experts] = None) -> dict:
+    """moe_forward on a ``synth.HostInputs``; ``rows`` selects a token subset. With ``fp8``
+    the routed experts are that FP8 bank (dequantised); the rest of the layer is unchanged."""
     x = inp.x if rows is None else inp.x[np.asarray(rows)]
-    return moe_forward(x, inp.w_router, inp.router_bias, inp.gate_up, inp.down,
+    gu, dn = (fp8.gate_up, fp8.down) if fp8 is not None else (inp.gate_up, inp.down)
+    return moe_forward(x, inp.w_router, inp.router_bias, gu, dn,
                        inp.ws_gate_up, inp.ws_down, inp.w_shared_gate, inp.cfg.k,
                        forced_ids=forced_ids)
