@@ -47,6 +47,8 @@ KERNEL_SOURCES = {  # kernel id -> source file whose hash a stored ncu traffic f
     "router_topk": ("router.cu",),
     "permute": ("permute.cu",),
     "combine": ("combine.cu",),
+    "gate_up_fp8": ("tc8_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
+    "down_fp8": ("tc8_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
 }
 # oracle token sample per workload for the CPU baseline (about 10-30 s on a host)
 CPU_SAMPLE = {"tiny": 64, "flash_decode": 16, "flash_prefill": 32, "flash_prefill_e64": 32,
@@ -126,9 +128,14 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- roofline
 
-def algorithmic_bytes(kernel: str, cfg, n_active: int) -> float:
-    """Bytes a launch of `kernel` must move at least (each operand once)."""
+def algorithmic_bytes(kernel: str, cfg, n_active: int, fp8: bool = False) -> float:
+    """Bytes a launch of `kernel` must move at least (each operand once). fp8: the routed
+    experts as E4M3 codes (1 byte per weight) plus one fp32 scale per weight row."""
     T, H, I, Is, R = cfg.T, cfg.H, cfg.I, cfg.Is, cfg.R
+    if fp8 and kernel == "gate_up":
+        return n_active * 2 * I * (H + 4) + (2 * Is * H + T * H) * 2 + (R * I + T * Is) * 4
+    if fp8 and kernel == "down":
+        return n_active * H * (I + 4) + H * Is * 2 + (R * I + T * Is) * 4 + T * H * 4
     if kernel == "gate_up":  # activated experts' gate|up + shared gate|up + x + h (hi+lo bf16)
         return (n_active * 2 * I * H + 2 * Is * H + T * H) * 2 + (R * I + T * Is) * 4
     if kernel == "down":  # activated experts' down + shared down + h (hi+lo) in + out (fp32)
@@ -184,8 +191,9 @@ def source_hash(kernel: str) -> str:
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def oracle_sample(cfg, seed: int, ntok: int):
-    """Inputs for timing the oracle on `ntok` sampled tokens (weights made beforehand)."""
+def oracle_sample(cfg, seed: int, ntok: int, fp8: bool = False):
+    """Inputs for timing the oracle on `ntok` sampled tokens (weights made beforehand; with
+    fp8, the routed experts quantised and dequantised as the FP8 layer uses them)."""
     import numpy as np
 
     import oracle
@@ -197,8 +205,9 @@ def oracle_sample(cfg, seed: int, ntok: int):
     x = host.x[rows]
     logits = oracle.router_logits(x, host.w_router, host.router_bias)
     ids, _ = oracle.topk_select(logits, cfg.k)
-    gu = {int(e): host.gate_up(int(e)) for e in np.unique(ids)}
-    dn = {int(e): host.down(int(e)) for e in np.unique(ids)}
+    src = oracle.Fp8Experts(host.gate_up, host.down) if fp8 else host
+    gu = {int(e): src.gate_up(int(e)) for e in np.unique(ids)}
+    dn = {int(e): src.down(int(e)) for e in np.unique(ids)}
     return host, x, gu, dn, rows
 
 
@@ -221,13 +230,14 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(cfg, seed=0):
+def cpu_baseline(cfg, seed=0, fp8=False):
     ntok = CPU_SAMPLE.get(cfg.name, 8)
-    host, x, gu, dn, rows = oracle_sample(cfg, seed, ntok)
+    host, x, gu, dn, rows = oracle_sample(cfg, seed, ntok, fp8)
     dt = time_oracle(cfg, host, x, gu, dn)
     return {"value": len(rows) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{len(rows)} of {cfg.T} tokens of the {cfg.name} layer (seed {seed}), full layer per "
-                      f"token in fp64; expert weights made before timing", "seconds": dt}
+                      f"token in fp64; expert weights made{' (FP8, dequantised)' if fp8 else ''} "
+                      f"before timing", "seconds": dt}
 
 
 # --------------------------------------------------------------------------- arms
@@ -334,19 +344,49 @@ def run_ours(args, cfg, world, rank, local):
         cfg = cfg.replace(I=I_c)
         torch.cuda.empty_cache()
     s = moe.shape_of(cfg)
+    fp8 = None
+    if args.fp8:
+        # weight pre-pass (once, at load time): routed experts to E4M3 codes + fp32 row
+        # scales; the bf16 routed banks are then freed (the FP8 layer does not read them)
+        t0 = time.time()
+        q = moe.quantize_fp8_experts(s, dev)
+        torch.cuda.synchronize()
+        fp8 = {"expert_weights": "E4M3 codes, one fp32 scale per weight row (amax/448)",
+               "shared_expert_and_router": "bf16 / fp32", "prepass_s": round(time.time() - t0, 3)}
+        dev["w_gate_up"] = None
+        dev["w_down"] = None
+        torch.cuda.empty_cache()
+        qs = moe.make_fp8_experts(q)
     ws = moe.alloc_workspace(s, host_staging=True)
     out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
     ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
     w = moe.make_weights(dev)
 
-    moe.moe_layer_forward(s, dev["x"], w, out, ws, topk_ids=ids)
+    def layer(x_dev, out_dev, topk_ids=None):
+        if fp8 is not None:
+            moe.moe_layer_forward_fp8(s, x_dev, w, qs, out_dev, ws, topk_ids=topk_ids)
+        else:
+            moe.moe_layer_forward(s, x_dev, w, out_dev, ws, topk_ids=topk_ids)
+
+    x_in = torch.empty_like(dev["x"])
+    out_in = torch.empty_like(out)
+
+    def layer_host(x_host, out_host):
+        if fp8 is not None:  # the same copies the host-buffer entry point makes
+            x_in.copy_(x_host, non_blocking=True)
+            layer(x_in, out_in)
+            out_host.copy_(out_in, non_blocking=True)
+        else:
+            moe.moe_layer_forward_host(s, x_host, w, out_host, ws)
+
+    layer(dev["x"], out, topk_ids=ids)
     st, flags = moe.moe_device_status(ws)
     if st != moe.MOE_OK:
         raise RuntimeError(f"device status {st} ({flags})")
     n_active = int(np.unique(ids.cpu().numpy()).size)
     for _ in range(args.warmup):
-        moe.moe_layer_forward(s, dev["x"], w, out, ws)
+        layer(dev["x"], out)
     torch.cuda.synchronize()
 
     props = torch.cuda.get_device_properties(local)
@@ -366,14 +406,14 @@ def run_ours(args, cfg, world, rank, local):
     windows = []
     graph = None
     moe.moe_profile_enable(True)  # fill the library's event pool before any capture
-    moe.moe_layer_forward(s, dev["x"], w, out, ws)
+    layer(dev["x"], out)
     torch.cuda.synchronize()
     moe.moe_profile_collect()
     if not args.no_graph:
         graph = torch.cuda.CUDAGraph()
         n_cap = moe.moe_launch_count()
         with torch.cuda.graph(graph, capture_error_mode="thread_local"):
-            moe.moe_layer_forward(s, dev["x"], w, out, ws)
+            layer(dev["x"], out)
         per_step = moe.moe_launch_count() - n_cap
         stream = torch.cuda.current_stream()
         for _ in range(2):
@@ -389,7 +429,7 @@ def run_ours(args, cfg, world, rank, local):
         if graph is not None:
             graph.replay()
         else:
-            moe.moe_layer_forward(s, dev["x"], w, out, ws)
+            layer(dev["x"], out)
     e1.record(stream)
     torch.cuda.synchronize()
     windows.append((w0, time.time()))
@@ -399,7 +439,7 @@ def run_ours(args, cfg, world, rank, local):
         # (the same kernels on the same data; events inside a graph cannot be timed)
         moe.moe_profile_collect()
         for _ in range(min(args.steps, 50)):
-            moe.moe_layer_forward(s, dev["x"], w, out, ws)
+            layer(dev["x"], out)
         torch.cuda.synchronize()
     moe.moe_profile_enable(False)
     prof = moe.moe_profile_collect()
@@ -413,13 +453,13 @@ def run_ours(args, cfg, world, rank, local):
     x_host = dev["x"].cpu().pin_memory()
     out_host = torch.empty((cfg.T, cfg.H), dtype=torch.float32).pin_memory()
     for _ in range(max(1, min(args.warmup, 3))):
-        moe.moe_layer_forward_host(s, x_host, w, out_host, ws)
+        layer_host(x_host, out_host)
     torch.cuda.synchronize()
     barrier()
     w0 = time.time()
     e0.record(stream)
     for _ in range(args.steps):
-        moe.moe_layer_forward_host(s, x_host, w, out_host, ws)
+        layer_host(x_host, out_host)
     e1.record(stream)
     torch.cuda.synchronize()
     windows.append((w0, time.time()))
@@ -442,27 +482,30 @@ def run_ours(args, cfg, world, rank, local):
         if v[1] > 0:
             kernels[k]["share"] = v[0] / tot
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
-    bound = "tensor" if kernel_flops(dom, cfg) / max(algorithmic_bytes(dom, cfg, n_active), 1) > 290 else "hbm"
+    is8 = fp8 is not None
+    dom_bytes = algorithmic_bytes(dom, cfg, n_active, is8)
+    bound = "tensor" if kernel_flops(dom, cfg) / max(dom_bytes, 1) > 290 else "hbm"
     per_launch_s = kernels[dom]["ms_per_launch"] / 1e3
     if bound == "hbm":
-        achieved = algorithmic_bytes(dom, cfg, n_active) / per_launch_s / 1e9
+        achieved = dom_bytes / per_launch_s / 1e9
         peak, unit = peaks["hbm_gbs"], "GB/s"
     else:
         achieved = kernel_flops(dom, cfg) / per_launch_s / 1e12
         peak, unit = peaks["bf16_tflops"], "TFLOP/s"
     roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
-                "algorithmic_bytes_per_launch": algorithmic_bytes(dom, cfg, n_active),
+                "algorithmic_bytes_per_launch": dom_bytes,
                 "activated_experts": n_active,
-                "traffic": stored_traffic(dom, cfg.name)}
+                "traffic": stored_traffic(dom + ("_fp8" if is8 else ""), cfg.name)}
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "us_per_layer": 1e3 * ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random router)",
-            "config": config_block(cfg, args.variant,
+            "config": config_block(cfg, "fp8" if args.fp8 else args.variant,
                                    "host launches of one layer forward per step" if args.no_graph
                                    else "CUDA graph replay of one layer forward per step"),
             "zero_channel_compaction": compact,
+            "fp8_experts": fp8,
             "roofline": roofline,
             "graph": not args.no_graph,
             "e2e": {"value": job_value(cfg.T, args.steps, world, ms_e2e), "unit": "tokens/s",
@@ -470,7 +513,7 @@ def run_ours(args, cfg, world, rank, local):
             "gpu_launches": launches, "kernels": kernels,
             "clocks": sampler.summary(windows) if sampler else None}
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(full_cfg if compact else cfg)
+        line["cpu_baseline"] = cpu_baseline(full_cfg if compact else cfg, fp8=fp8 is not None)
     return line
 
 
@@ -486,6 +529,8 @@ def main():
     ap.add_argument("--variant", default="auto", choices=["auto", "stream", "tc", "tc2"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel from the host")
+    ap.add_argument("--fp8", action="store_true",
+                    help="routed experts in FP8 (E4M3 + fp32 row scales, quantised before timing)")
     ap.add_argument("--compact", action="store_true",
                     help="zero-channel compaction of the routed experts before timing (weight pre-pass)")
     args = ap.parse_args()

@@ -238,6 +238,45 @@ moe_status moe_compact_zero_channels(const moe_shape* shape, const void* w_gate_
                                      const void* w_down, int32_t I_c, void* gate_up_c,
                                      void* down_c, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * FP8 routed experts. Source: "Qwen3.8, weights in hand: 98% of a 2.4T model is routed
+ * experts", section "What FP8 actually quantizes". The FP8 checkpoint stores the routed
+ * experts at one byte per parameter and keeps the router, the shared expert and the
+ * shared-expert gate in bf16. The page does not name the 8-bit format or its scaling; this
+ * library reads it as E4M3 codes (bias 7, largest finite 448, 0x7F/0xFF NaN) with one fp32
+ * scale per weight row:
+ *   scale = amax_row / 448 (fp32 division; 0 for an all-zero row)
+ *   code  = E4M3 round-to-nearest-even of (w / scale) (fp32 division), clamped to +-448
+ * and the weight the layer uses is decode(code) * scale. Activations, h and the output
+ * keep the precision of the bf16 layer.
+ *
+ * moe_fp8_experts: q_gate_up uint8 [E][2I][H] (rows 0..I-1 gate, I..2I-1 up), s_gate_up
+ *   fp32 [E][2I], q_down uint8 [E][H][I], s_down fp32 [E][H]. Device pointers, 16-byte
+ *   aligned, caller-owned.
+ * moe_quantize_fp8_experts: the weight pre-pass (run once at load time), bf16 w_gate_up
+ *   [E][2I][H] and w_down [E][H][I] -> the four arrays above; asynchronous on `stream`.
+ *   Errors: MOE_ERR_INVALID_ARG (null or misaligned pointer), MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA.
+ * moe_layer_forward_fp8: moe_layer_forward with the routed experts taken from `experts`
+ *   (weights->w_gate_up and weights->w_down are not read and may be NULL). Supported for
+ *   decode-size batches, T*k < 16*E, with I and Is multiples of 128 and H of 256 on
+ *   sm_100; otherwise MOE_ERR_UNSUPPORTED. Same outputs, workspace and errors as
+ *   moe_layer_forward.
+ */
+typedef struct moe_fp8_experts {
+  const void* q_gate_up;
+  const float* s_gate_up;
+  const void* q_down;
+  const float* s_down;
+} moe_fp8_experts;
+
+moe_status moe_quantize_fp8_experts(const moe_shape* shape, const void* w_gate_up,
+                                    const void* w_down, void* q_gate_up, float* s_gate_up,
+                                    void* q_down, float* s_down, void* stream);
+moe_status moe_layer_forward_fp8(const moe_shape* shape, const void* x,
+                                 const moe_weights* weights, const moe_fp8_experts* experts,
+                                 float* out, int32_t* topk_ids, float* topk_w, float* gap,
+                                 void* ws, size_t ws_bytes, void* stream);
+
 /* Choose the grouped-GEMM variant for later calls (process-wide; default AUTO). */
 moe_status moe_set_variant(moe_variant variant);
 

@@ -11,7 +11,7 @@ codes into exceptions. There is no CPU path: if the library is missing, importin
 package raises.
 
 Names follow the C ABI: moe_router_topk, moe_permute, moe_grouped_swiglu,
-moe_unpermute_combine, moe_layer_forward, moe_layer_forward_host, ...
+moe_unpermute_combine, moe_layer_forward, moe_layer_forward_host, moe_layer_forward_fp8, ...
 """
 from __future__ import annotations
 
@@ -54,6 +54,10 @@ class moe_weights(ctypes.Structure):
                                                "ws_gate_up", "ws_down", "w_shared_gate")]
 
 
+class moe_fp8_experts(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("q_gate_up", "s_gate_up", "q_down", "s_down")]
+
+
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
                       "`python sparse_moe_expert_fp32_b200/build.py` (nvcc, sm_100a)")
@@ -62,6 +66,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 _vp, _sz, _i32, _u64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_uint64
 _SP = ctypes.POINTER(moe_shape)
 _WP = ctypes.POINTER(moe_weights)
+_FP = ctypes.POINTER(moe_fp8_experts)
 
 _SIGS = {
     "moe_workspace_bytes": ([_SP], _sz),
@@ -74,6 +79,9 @@ _SIGS = {
     "moe_unpermute_combine": ([_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moe_layer_forward": ([_SP, _vp, _WP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_layer_forward_host": ([_SP, _vp, _WP, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_quantize_fp8_experts": ([_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moe_layer_forward_fp8": ([_SP, _vp, _WP, _FP, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+                              ctypes.c_int),
     "moe_set_variant": ([ctypes.c_int], ctypes.c_int),
     "moe_compact_workspace_bytes": ([_SP], _sz),
     "moe_zero_channel_count": ([_SP, _vp, ctypes.POINTER(ctypes.c_int32), _vp, _sz, _vp], ctypes.c_int),
@@ -143,6 +151,12 @@ def make_weights(w: dict) -> moe_weights:
     return moe_weights(_ptr(w["w_router"]), _ptr(w.get("router_bias")), _ptr(w["w_gate_up"]),
                        _ptr(w["w_down"]), _ptr(w["ws_gate_up"]), _ptr(w["ws_down"]),
                        _ptr(w["w_shared_gate"]))
+
+
+def make_fp8_experts(q: dict) -> moe_fp8_experts:
+    """moe_fp8_experts from a dict of device tensors keyed like the C struct."""
+    return moe_fp8_experts(_ptr(q["q_gate_up"]), _ptr(q["s_gate_up"]), _ptr(q["q_down"]),
+                           _ptr(q["s_down"]))
 
 
 def _w(weights) -> moe_weights:
@@ -239,6 +253,24 @@ def moe_compact_zero_channels(shape, w_gate_up, w_down, I_c, gate_up_c, down_c, 
            "moe_compact_zero_channels")
 
 
+def moe_quantize_fp8_experts(shape, w_gate_up, w_down, q_gate_up, s_gate_up, q_down, s_down,
+                             stream=None):
+    _check(_lib.moe_quantize_fp8_experts(ctypes.byref(shape), _ptr(w_gate_up), _ptr(w_down),
+                                         _ptr(q_gate_up), _ptr(s_gate_up), _ptr(q_down),
+                                         _ptr(s_down), _stream(stream)),
+           "moe_quantize_fp8_experts")
+
+
+def moe_layer_forward_fp8(shape, x, weights, experts, out, ws, topk_ids=None, topk_w=None,
+                          gap=None, stream=None):
+    w = _w(weights)
+    q = experts if isinstance(experts, moe_fp8_experts) else make_fp8_experts(experts)
+    _check(_lib.moe_layer_forward_fp8(ctypes.byref(shape), _ptr(x), ctypes.byref(w),
+                                      ctypes.byref(q), _ptr(out), _ptr(topk_ids), _ptr(topk_w),
+                                      _ptr(gap), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "moe_layer_forward_fp8")
+
+
 def moe_set_variant(variant: int) -> None:
     _check(_lib.moe_set_variant(int(variant)), "moe_set_variant")
 
@@ -307,3 +339,20 @@ def compact_zero_channels(shape: moe_shape, weights: dict, multiple: int = 128, 
     out["w_gate_up"] = gu
     out["w_down"] = dn
     return out, I_c
+
+
+def quantize_fp8_experts(shape: moe_shape, weights: dict, stream=None) -> dict:
+    """The FP8 expert pre-pass on a weight dict (run once): allocates and returns
+    {q_gate_up uint8 [E][2I][H], s_gate_up fp32 [E][2I], q_down uint8 [E][H][I],
+    s_down fp32 [E][H]} on the routed banks' device."""
+    import torch
+
+    E, H, I = shape.E, shape.H, shape.I
+    d = weights["w_gate_up"].device
+    q = {"q_gate_up": torch.empty((E, 2 * I, H), dtype=torch.uint8, device=d),
+         "s_gate_up": torch.empty((E, 2 * I), dtype=torch.float32, device=d),
+         "q_down": torch.empty((E, H, I), dtype=torch.uint8, device=d),
+         "s_down": torch.empty((E, H), dtype=torch.float32, device=d)}
+    moe_quantize_fp8_experts(shape, weights["w_gate_up"], weights["w_down"], q["q_gate_up"],
+                             q["s_gate_up"], q["q_down"], q["s_down"], stream)
+    return q

@@ -384,6 +384,68 @@ moe_status moe_compact_zero_channels(const moe_shape* shape, const void* w_gate_
   return MOE_OK;
 }
 
+moe_status moe_quantize_fp8_experts(const moe_shape* shape, const void* w_gate_up,
+                                    const void* w_down, void* q_gate_up, float* s_gate_up,
+                                    void* q_down, float* s_down, void* stream) {
+  MOE_TRY(check_shape(shape));
+  const moe_shape& s = *shape;
+  if (!aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(q_gate_up) ||
+      !aligned16(s_gate_up) || !aligned16(q_down) || !aligned16(s_down))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  int dev = 0, sms = 148;
+  MOE_CUDA(cudaGetDevice(&dev));
+  MOE_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  MOE_CUDA(launch_quantize_fp8_rows(static_cast<const uint16_t*>(w_gate_up),
+                                    (size_t)s.E * 2 * s.I, s.H, static_cast<uint8_t*>(q_gate_up),
+                                    s_gate_up, sms, st));
+  MOE_CUDA(launch_quantize_fp8_rows(static_cast<const uint16_t*>(w_down), (size_t)s.E * s.H, s.I,
+                                    static_cast<uint8_t*>(q_down), s_down, sms, st));
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward_fp8(const moe_shape* shape, const void* x, const moe_weights* weights,
+                                 const moe_fp8_experts* experts, float* out, int32_t* topk_ids,
+                                 float* topk_w, float* gap, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  MOE_TRY(check_shape(shape));
+  const moe_shape& s = *shape;
+  MOE_TRY(check_router_weights(weights));
+  if (!aligned16(weights->ws_gate_up) || !aligned16(weights->ws_down)) return MOE_ERR_INVALID_ARG;
+  if (!experts || !aligned16(experts->q_gate_up) || !aligned16(experts->s_gate_up) ||
+      !aligned16(experts->q_down) || !aligned16(experts->s_down))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if ((topk_ids && !aligned16(topk_ids)) || (topk_w && !aligned16(topk_w)) ||
+      (gap && !aligned16(gap)))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(s, ws, ws_bytes));
+  if (s.T == 0) return MOE_OK;
+  if (!tc8_supported(s)) return MOE_ERR_UNSUPPORTED;
+  const Layout L = layout(s);
+  char* w = static_cast<char*>(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  int32_t* ids = topk_ids ? topk_ids : reinterpret_cast<int32_t*>(w + L.ids);
+  float* tw = topk_w ? topk_w : reinterpret_cast<float*>(w + L.w);
+  float* sg = reinterpret_cast<float*>(w + L.sgate);
+  float* logits = reinterpret_cast<float*>(w + L.logits);
+  int32_t* sorted_token = reinterpret_cast<int32_t*>(w + L.sorted_token);
+  float* sorted_w = reinterpret_cast<float*>(w + L.sorted_w);
+
+  MOE_CUDA(launch_router_logits(s, L, w, xb, weights->w_router, logits, st));
+  MOE_CUDA(launch_router_topk(s, logits, weights->w_router, weights->router_bias, xb,
+                              static_cast<const uint16_t*>(weights->w_shared_gate), ids, tw, sg,
+                              gap, out /* rows zeroed here, accumulated by the down GEMM */, st));
+  MOE_CUDA(launch_permute(s, L, w, ids, tw, reinterpret_cast<int32_t*>(w + L.offsets),
+                          sorted_token, sorted_w, reinterpret_cast<int32_t*>(w + L.assign_row),
+                          st));
+  MOE_CUDA(launch_tc8_gate_up(s, L, w, xb, sorted_token, *weights, *experts, st));
+  MOE_CUDA(launch_tc8_down(s, L, w, sorted_token, sorted_w, sg, *weights, *experts, nullptr,
+                           nullptr, out, st));
+  return MOE_OK;
+}
+
 moe_status moe_set_variant(moe_variant variant) {
   if (variant != MOE_VARIANT_AUTO && variant != MOE_VARIANT_STREAM && variant != MOE_VARIANT_TC &&
       variant != MOE_VARIANT_TC2)

@@ -130,6 +130,9 @@ cudaError_t launch_zero_channel_map(const moe_shape& s, const uint16_t* w_gate_u
 cudaError_t launch_compact_banks(const moe_shape& s, const uint16_t* w_gate_up,
                                  const uint16_t* w_down, const int32_t* src, int Ic,
                                  uint16_t* gate_up_c, uint16_t* down_c, cudaStream_t st);
+// FP8 expert pre-pass (fp8_quant.cu): rows of n bf16 -> E4M3 codes and fp32 row scales.
+cudaError_t launch_quantize_fp8_rows(const uint16_t* w, size_t rows, int n, uint8_t* q,
+                                     float* scale, int sms, cudaStream_t st);
 cudaError_t launch_wait_flag(const int32_t* flag, uint64_t timeout_ns, uint32_t* status,
                              cudaStream_t st);
 

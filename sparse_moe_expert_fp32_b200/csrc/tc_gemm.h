@@ -34,4 +34,16 @@ cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
                             const moe_weights& w, float* y, float* y_shared, float* out,
                             cudaStream_t st);
 
+// The same grouped GEMMs with the routed experts' weights in FP8 (E4M3 codes, one fp32 scale
+// per weight row; the shared expert stays bf16): one CTA per tile, codes widened to bf16 in
+// shared memory. Decode-size batches only (T*k < 16*E), on tensor-core shapes.
+bool tc8_supported(const moe_shape& s);
+cudaError_t launch_tc8_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
+                               const int32_t* sorted_token, const moe_weights& w,
+                               const moe_fp8_experts& q, cudaStream_t st);
+cudaError_t launch_tc8_down(const moe_shape& s, const Layout& L, char* ws,
+                            const int32_t* sorted_token, const float* sorted_w, const float* sgate,
+                            const moe_weights& w, const moe_fp8_experts& q, float* y,
+                            float* y_shared, float* out, cudaStream_t st);
+
 }  // namespace moe

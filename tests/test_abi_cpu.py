@@ -112,3 +112,35 @@ def test_profile_collect_empty():
     r = moe.moe_profile_collect()
     assert set(r) == set(moe.KERNELS)
     assert all(v == (0.0, 0) for v in r.values())
+
+
+def test_fp8_entry_points_reject_bad_pointers_before_launch():
+    s = moe.shape_of(synth.CONFIGS["tiny"], T=32)
+    L = moe.lib()
+    w = moe.moe_weights(16, 0, 0, 0, 64, 80, 96)  # routed bf16 banks unused: NULL is allowed
+    q = moe.moe_fp8_experts(4096, 8192, 12288, 16384)
+    before = moe.moe_launch_count()
+    # no FP8 bank
+    assert L.moe_layer_forward_fp8(ctypes.byref(s), 16, ctypes.byref(w), None, 16, None, None,
+                                   None, 4096, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    # misaligned scale array
+    q2 = moe.moe_fp8_experts(4096, 8196, 12288, 16384)
+    assert L.moe_layer_forward_fp8(ctypes.byref(s), 16, ctypes.byref(w), ctypes.byref(q2), 16,
+                                   None, None, None, 4096, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    # shared expert missing
+    w2 = moe.moe_weights(16, 0, 0, 0, 0, 80, 96)
+    assert L.moe_layer_forward_fp8(ctypes.byref(s), 16, ctypes.byref(w2), ctypes.byref(q), 16,
+                                   None, None, None, 4096, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    # workspace too small
+    assert L.moe_layer_forward_fp8(ctypes.byref(s), 16, ctypes.byref(w), ctypes.byref(q), 16,
+                                   None, None, None, 4096, 1024, None) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    # empty batch: nothing launched
+    s0 = moe.shape_of(synth.CONFIGS["tiny"], T=0)
+    assert L.moe_layer_forward_fp8(ctypes.byref(s0), 16, ctypes.byref(w), ctypes.byref(q), 16,
+                                   None, None, None, 4096, 1 << 30, None) == moe.MOE_OK
+    # the pre-pass
+    assert L.moe_quantize_fp8_experts(ctypes.byref(s), 16, None, 32, 48, 64, 80,
+                                      None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_fp8_experts(ctypes.byref(s), 16, 32, 48, 64, 80, 100,
+                                      None) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_launch_count() == before

@@ -58,3 +58,13 @@ def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
     assert bench.source_hash("down") == h0
     p.write_text(src.replace("kSlotCols = 256", "kSlotCols = 255", 1))
     assert bench.source_hash("down") != h0
+
+
+def test_decode_fp8_bytes_by_hand():
+    # the FP8 layer: routed gate|up and down weights at one byte each plus one fp32 scale per
+    # weight row; the shared expert, x, h and out as in the bf16 layer
+    cfg = synth.CONFIGS["flash_decode"]
+    gu = 370 * 2 * 640 * (2560 + 4) + (2 * 640 * 2560 + 64 * 2560) * 2 + (640 * 640 + 64 * 640) * 4
+    dn = 370 * 2560 * (640 + 4) + 2560 * 640 * 2 + (640 * 640 + 64 * 640) * 4 + 64 * 2560 * 4
+    assert bench.algorithmic_bytes("gate_up", cfg, 370, fp8=True) == gu == 1222993920
+    assert bench.algorithmic_bytes("down", cfg, 370, fp8=True) == dn == 615731200

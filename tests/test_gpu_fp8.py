@@ -1,0 +1,199 @@
+"""GPU parity of the FP8 routed-expert path through the C ABI.
+
+Source: "Qwen3.8, weights in hand: 98% of a 2.4T model is routed experts", section "What
+FP8 actually quantizes" (routed experts in FP8; router, shared expert and its gate bf16).
+Reading: E4M3 codes with one fp32 scale per weight row (scale = amax / 448), stated in
+include/moe.h and in the oracle.
+
+* The pre-pass (moe_quantize_fp8_experts) takes every rounding decision in fp32 on both
+  sides, so its codes and scales must equal the oracle's bit for bit.
+* The layer (moe_layer_forward_fp8) must match the fp64 oracle evaluated on the
+  dequantised FP8 bank within the layer tolerance (the FP8 rounding is part of the model,
+  not of the error): decode-size batches, several tile geometries, zero rows, rows whose
+  codes are nearly all E4M3 subnormals, and the Flash-Next decode layer at full size in the
+  configuration `bench.py --fp8` times.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU, skipped there
+    pytestmark = pytest.mark.skip(reason="needs a CUDA device")
+
+import oracle  # noqa: E402
+import sparse_moe_expert_fp32_b200 as moe  # noqa: E402
+import synth  # noqa: E402
+from parity_util import assert_layer_close, id_sets_match  # noqa: E402
+
+TINY = synth.CONFIGS["tiny"]
+CASES = {
+    # T*k < 16*E in every case: the FP8 path serves decode-size batches
+    "tiny_T48": dict(T=48),
+    "T1": dict(T=1),
+    "T3_ragged": dict(T=3),
+    "E1": dict(T=8, E=1, k=1),
+    "zero_rows": dict(T=48, zero_rows_pct=50),
+    "shared_narrower": dict(T=40, I=256, Is=128),
+}
+
+
+def _u16(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _dev_bf16(u16):
+    return torch.from_numpy(np.ascontiguousarray(u16).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _quantize(cfg, dev):
+    q = moe.quantize_fp8_experts(moe.shape_of(cfg), dev)
+    torch.cuda.synchronize()
+    return q
+
+
+def _forward_fp8(cfg, dev, q):
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s)
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    w = dict(dev)
+    w["w_gate_up"] = None  # the FP8 layer does not read the bf16 routed banks
+    w["w_down"] = None
+    moe.moe_layer_forward_fp8(s, dev["x"], w, q, out, ws, topk_ids=ids)
+    st, flags = moe.moe_device_status(ws)
+    assert st == moe.MOE_OK, (st, flags)
+    return out.cpu().numpy(), ids.cpu().numpy()
+
+
+def _check(cfg, host, fp8, out, ids, rows):
+    ref = oracle.forward_inputs(host, rows=rows, fp8=fp8)
+    differ = id_sets_match(ids[rows], ref["ids"], ref["gap"], ref["logits"])
+    keep = [i for i in range(len(rows)) if i not in set(differ)]
+    return assert_layer_close(out[rows][keep], ref["out"][keep], cfg.name), len(differ)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", ["tiny_T48", "zero_rows"])
+def test_quantize_bitexact(case):
+    cfg = TINY.replace(name=case, **CASES[case])
+    dev = synth.device_inputs(cfg, seed=2)
+    host = synth.host_inputs(cfg, seed=2)
+    q = _quantize(cfg, dev)
+    for e in range(cfg.E):
+        c, s = oracle.quantize_fp8_rows(host.gate_up(e))
+        assert np.array_equal(q["q_gate_up"][e].cpu().numpy(), c), e
+        assert np.array_equal(q["s_gate_up"][e].cpu().numpy().view(np.uint32), s.view(np.uint32)), e
+        c, s = oracle.quantize_fp8_rows(host.down(e))
+        assert np.array_equal(q["q_down"][e].cpu().numpy(), c), e
+        assert np.array_equal(q["s_down"][e].cpu().numpy().view(np.uint32), s.view(np.uint32)), e
+    if cfg.zero_rows_pct:
+        assert (q["s_gate_up"] == 0).any()
+
+
+@pytest.mark.gpu
+def test_quantize_bitexact_flash_decode_experts():
+    cfg = synth.CONFIGS["flash_decode"]
+    dev = synth.device_inputs(cfg, seed=0)
+    host = synth.host_inputs(cfg, seed=0)
+    q = _quantize(cfg, dev)
+    for e in (0, 1, 255, 511):
+        c, s = oracle.quantize_fp8_rows(host.gate_up(e))
+        assert np.array_equal(q["q_gate_up"][e].cpu().numpy(), c), e
+        assert np.array_equal(q["s_gate_up"][e].cpu().numpy().view(np.uint32), s.view(np.uint32)), e
+        c, s = oracle.quantize_fp8_rows(host.down(e))
+        assert np.array_equal(q["q_down"][e].cpu().numpy(), c), e
+        assert np.array_equal(q["s_down"][e].cpu().numpy().view(np.uint32), s.view(np.uint32)), e
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_fp8_layer_small(case):
+    cfg = TINY.replace(name=case, **CASES[case])
+    assert cfg.T * cfg.k < 16 * cfg.E
+    dev = synth.device_inputs(cfg, seed=4)
+    host = synth.host_inputs(cfg, seed=4)
+    q = _quantize(cfg, dev)
+    out, ids = _forward_fp8(cfg, dev, q)
+    fp8 = oracle.Fp8Experts(host.gate_up, host.down)
+    stats, ties = _check(cfg, host, fp8, out, ids, list(range(cfg.T)))
+    print(case, stats, "near-ties", ties)
+
+
+@pytest.mark.gpu
+def test_fp8_layer_hot_expert_several_tiles():
+    """Every token on expert 7: 200 routed rows in one group (four 64-row gate|up tiles, two
+    112-row down tiles that take both TMEM slots) and 200 shared rows."""
+    cfg = TINY.replace(name="hot_decode", T=200, E=256, k=4)
+    assert cfg.T * cfg.k < 16 * cfg.E
+    dev = synth.device_inputs(cfg, seed=8)
+    bias = np.zeros(cfg.E, np.float32)
+    bias[7] = 50.0
+    dev["router_bias"] = torch.from_numpy(bias).cuda()
+    host = synth.host_inputs(cfg, seed=8)
+    host.router_bias = bias
+    q = _quantize(cfg, dev)
+    out, ids = _forward_fp8(cfg, dev, q)
+    assert (ids == 7).any(axis=1).all()
+    fp8 = oracle.Fp8Experts(host.gate_up, host.down)
+    _check(cfg, host, fp8, out, ids, list(range(cfg.T)))
+
+
+@pytest.mark.gpu
+def test_fp8_layer_subnormal_codes():
+    """Every routed weight row gets one outlier (640) in column 0, so its scale is 640/448
+    and nearly all its other codes are E4M3 subnormals (|w / scale| < 2^-6). Column 0 of x
+    is zeroed and gate row 0 of every expert too (h_0 = 0), so the outliers add nothing and
+    the output comes from the small codes alone: widening them wrongly (flushed to zero, a
+    wrong exponent) cannot hide behind the outliers."""
+    cfg = TINY.replace(name="subnormal", T=48)
+    dev = synth.device_inputs(cfg, seed=9)
+    host = synth.host_inputs(cfg, seed=9)
+    gu, dn = host.gate_up_all(), host.down_all()
+    big = np.uint16(0x4420)  # 640.0 in bf16
+    gu[:, :, 0] = big
+    gu[:, 0, :] = 0
+    dn[:, :, 0] = big
+    host.x[:, 0] = 0
+    dev["w_gate_up"] = _dev_bf16(gu)
+    dev["w_down"] = _dev_bf16(dn)
+    dev["x"] = _dev_bf16(host.x)
+    q = _quantize(cfg, dev)
+    codes = q["q_gate_up"][:, 1:, 1:].cpu().numpy()
+    assert ((codes & 0x78) == 0).mean() > 0.5  # most codes are subnormal (or zero)
+    out, ids = _forward_fp8(cfg, dev, q)
+    fp8 = oracle.Fp8Experts(lambda e: gu[e], lambda e: dn[e])
+    stats, _ = _check(cfg, host, fp8, out, ids, list(range(cfg.T)))
+    print("subnormal", stats)
+
+
+@pytest.mark.gpu
+def test_fp8_layer_flash_decode_sampled():
+    """The Flash-Next decode layer at full size (T=64, E=512, k=10, I=640), as timed."""
+    cfg = synth.CONFIGS["flash_decode"]
+    dev = synth.device_inputs(cfg, seed=0)
+    q = _quantize(cfg, dev)
+    out, ids = _forward_fp8(cfg, dev, q)
+    del dev, q
+    torch.cuda.empty_cache()
+    host = synth.host_inputs(cfg, seed=0)
+    fp8 = oracle.Fp8Experts(host.gate_up, host.down)
+    rng = np.random.default_rng(77)
+    rows = sorted(set([0, cfg.T - 1] + rng.choice(cfg.T, 10, replace=False).tolist()))
+    stats, ties = _check(cfg, host, fp8, out, ids, rows)
+    print("flash_decode fp8", stats, "near-ties", ties)
+
+
+@pytest.mark.gpu
+def test_fp8_rejects_prefill_size_batches():
+    cfg = synth.CONFIGS["flash_prefill"]  # T*k >= 16*E
+    s = moe.shape_of(cfg)
+    w = moe.moe_weights(16, 0, 0, 0, 64, 80, 96)
+    q = moe.moe_fp8_experts(4096, 8192, 12288, 16384)
+    ws = moe.alloc_workspace(moe.shape_of(cfg, T=1))  # any aligned pointer: nothing launches
+    before = moe.moe_launch_count()
+    st = moe.lib().moe_layer_forward_fp8(moe.ctypes.byref(s), 16, moe.ctypes.byref(w),
+                                         moe.ctypes.byref(q), 16, None, None, None, ws.data_ptr(),
+                                         moe.moe_workspace_bytes(s), None)
+    assert st == moe.MOE_ERR_UNSUPPORTED
+    assert moe.moe_launch_count() == before
