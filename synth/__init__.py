@@ -96,6 +96,10 @@ CONFIGS = {
         "flash_prefill_e64", T=1024, H=2560, E=64, k=10, I=640, Is=640,
         description="Flash-Next-shaped prefill with 64 experts: T=1024 (160 tokens per expert as at "
                     "T=8192 with 512 experts), 630 MB of expert weights; the profiling case"),
+    "flash_decode_e64": LayerConfig(
+        "flash_decode_e64", T=64, H=2560, E=64, k=10, I=640, Is=640,
+        description="Flash-Next-shaped decode with 64 experts: T=64 (10 tokens per expert), "
+                    "630 MB of bf16 expert weights, 315 MB in FP8; the FP8 profiling case"),
     "t24_prefill_e16": LayerConfig(
         "t24_prefill_e16", T=256, H=8192, E=16, k=10, I=2048, Is=2048,
         description="2.4T-shaped prefill with 16 experts: T=256 (160 tokens per expert as at "
