@@ -33,6 +33,12 @@ Readings of points the pages leave open (each listed in the design notes):
 * the shared-expert gate is a length-H bf16 vector without bias;
 * gate|up weights are one [2I][H] tensor per expert, gate rows first.
 
+FP8 routed experts (optional, section "FP8 experts" below): the routed banks quantised to
+E4M3 codes with one fp32 scale per weight row and dequantised exactly; the layer above then
+runs on those weights ("Qwen3.8, weights in hand: 98% of a 2.4T model is routed experts",
+section "What FP8 actually quantizes"; the format and scaling are readings, stated there).
+Pinned by tests/test_fp8_oracle.py.
+
 Parity status: values in general are "parity unpinned by the pages" (no worked numeric
 example of a layer output is printed); the pins are closed forms, special cases, brute
 force on tiny inputs and the pages' shape and parameter counts (tests/test_oracle_pins.py).
