@@ -290,7 +290,8 @@ def run_reference(args, cfg, world, rank):
     if rank != 0:
         return None
     ntok = CPU_SAMPLE.get(cfg.name, 8)
-    host, x, gu, dn, rows = oracle_sample(cfg, 0, ntok)
+    fp8 = bool(getattr(args, "fp8", False))
+    host, x, gu, dn, rows = oracle_sample(cfg, 0, ntok, fp8)
     for _ in range(args.warmup):
         time_oracle(cfg, host, x, gu, dn)
     total = 0.0
@@ -303,7 +304,7 @@ def run_reference(args, cfg, world, rank):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_block(cfg, None, "fp64 oracle on the host cores"),
+            "config": config_block(cfg, "fp8" if fp8 else None, "fp64 oracle on the host cores"),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -68,3 +68,17 @@ def test_decode_fp8_bytes_by_hand():
     dn = 370 * 2560 * (640 + 4) + 2560 * 640 * 2 + (640 * 640 + 64 * 640) * 4 + 64 * 2560 * 4
     assert bench.algorithmic_bytes("gate_up", cfg, 370, fp8=True) == gu == 1222993920
     assert bench.algorithmic_bytes("down", cfg, 370, fp8=True) == dn == 615731200
+
+
+def test_reference_arm_times_the_fp8_oracle():
+    import json
+    import subprocess
+    import sys
+
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--fp8", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, cwd=bench.ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][-1])
+    assert line["impl"] == "reference" and line["config"]["variant"] == "fp8"
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
