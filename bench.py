@@ -500,7 +500,8 @@ def run_ours(args, cfg, world, rank, local):
                 "traffic": stored_traffic(dom + ("_fp8" if is8 else ""), cfg.name)}
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "us_per_layer": 1e3 * ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 (gate|up MMAs), bf16 (down MMAs)" if fp8 is not None else "bf16",
             "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random router)",
             "config": config_block(cfg, "fp8" if args.fp8 else args.variant,
                                    "host launches of one layer forward per step" if args.no_graph
