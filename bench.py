@@ -364,9 +364,28 @@ def run_ours(args, cfg, world, rank, local):
     stream = torch.cuda.current_stream()
     w = moe.make_weights(dev)
 
+    if args.staged:
+        # the four stage entry points, y materialised in fp32 and combined by its own kernel
+        R = cfg.T * cfg.k
+        st_ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+        st_w = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device="cuda")
+        st_sg = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
+        st_off = torch.empty((cfg.E + 1,), dtype=torch.int32, device="cuda")
+        st_tok = torch.empty((R,), dtype=torch.int32, device="cuda")
+        st_ar = torch.empty((R,), dtype=torch.int32, device="cuda")
+        st_y = torch.empty((R, cfg.H), dtype=torch.float32, device="cuda")
+        st_ys = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+
     def layer(x_dev, out_dev, topk_ids=None):
         if fp8 is not None:
             moe.moe_layer_forward_fp8(s, x_dev, w, qs, out_dev, ws, topk_ids=topk_ids)
+        elif args.staged:
+            moe.moe_router_topk(s, x_dev, w, st_ids, st_w, st_sg, None, ws)
+            moe.moe_permute(s, st_ids, st_off, st_tok, st_ar, ws)
+            moe.moe_grouped_swiglu(s, x_dev, st_tok, st_off, w, st_y, st_ys, ws)
+            moe.moe_unpermute_combine(s, st_y, st_ys, st_ar, st_w, st_sg, out_dev)
+            if topk_ids is not None:
+                topk_ids.copy_(st_ids)
         else:
             moe.moe_layer_forward(s, x_dev, w, out_dev, ws, topk_ids=topk_ids)
 
@@ -374,7 +393,7 @@ def run_ours(args, cfg, world, rank, local):
     out_in = torch.empty_like(out)
 
     def layer_host(x_host, out_host):
-        if fp8 is not None:  # the same copies the host-buffer entry point makes
+        if fp8 is not None or args.staged:  # the copies the host-buffer entry point makes
             x_in.copy_(x_host, non_blocking=True)
             layer(x_in, out_in)
             out_host.copy_(out_in, non_blocking=True)
@@ -503,7 +522,8 @@ def run_ours(args, cfg, world, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 (gate|up MMAs), bf16 (down MMAs)" if fp8 is not None else "bf16",
             "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random router)",
-            "config": config_block(cfg, "fp8" if args.fp8 else args.variant,
+            "config": config_block(cfg, "fp8" if args.fp8 else
+                                   (args.variant + "+staged" if args.staged else args.variant),
                                    "host launches of one layer forward per step" if args.no_graph
                                    else "CUDA graph replay of one layer forward per step"),
             "zero_channel_compaction": compact,
@@ -531,6 +551,9 @@ def main():
     ap.add_argument("--variant", default="auto", choices=["auto", "stream", "tc", "tc2"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel from the host")
+    ap.add_argument("--staged", action="store_true",
+                    help="time the four stage entry points (y in fp32, separate combine) "
+                         "instead of the fused layer forward")
     ap.add_argument("--fp8", action="store_true",
                     help="routed experts in FP8 (E4M3 + fp32 row scales, quantised before timing)")
     ap.add_argument("--compact", action="store_true",
