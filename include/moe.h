@@ -151,9 +151,12 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_ids, int32_t*
  * routine. Limit: ceil(T/256) * E <= 16384 (for example T <= 8192 with E = 512); larger
  * shapes return MOE_ERR_UNSUPPORTED (use moe_permute with a workspace). The first call on
  * a device looks up the array's device address; make that first call before capturing a
- * stream into a CUDA graph. All calls share the one array: calls that overlap on the GPU
- * (different streams, or several host threads) race and give wrong results. An id outside
- * [0, E) is skipped; offsets[E] then falls short of T*k.
+ * stream into a CUDA graph. The address is kept until the process exits: do not call this
+ * after a cudaDeviceReset (or another teardown of the device's primary context) in the
+ * same process. All calls share the one array: calls that overlap on the GPU (different
+ * streams, or several host threads) race and give wrong results. An id outside [0, E) is
+ * skipped and not reported (the array's status word has no reader); offsets[E] then falls
+ * short of T*k, which the caller can check.
  */
 moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_ids, int32_t* offsets,
                                int32_t* sorted_token, int32_t* assign_row, void* stream);
@@ -277,8 +280,13 @@ moe_status moe_layer_forward_fp8(const moe_shape* shape, const void* x,
                                  float* out, int32_t* topk_ids, float* topk_w, float* gap,
                                  void* ws, size_t ws_bytes, void* stream);
 
-/* Choose the grouped-GEMM variant for later calls (process-wide; default AUTO). */
+/* Grouped-GEMM variant. moe_workspace_set_variant chooses it for the calls made with the
+ * workspace `ws` (its address is the key; moe_workspace_init clears the choice, so a new
+ * workspace allocated at a reused address starts from the default). moe_set_variant sets
+ * the process-wide default, used by workspaces without a choice of their own (initially
+ * AUTO). Both take effect at the next call; neither touches the GPU. */
 moe_status moe_set_variant(moe_variant variant);
+moe_status moe_workspace_set_variant(void* ws, size_t ws_bytes, moe_variant variant);
 
 /* Synchronise `stream`, read the workspace status word (MOE_OK, MOE_ERR_DEVICE_BOUNDS
  * or MOE_ERR_DEVICE_TIMEOUT), and clear it. `detail` (HOST, may be NULL) receives

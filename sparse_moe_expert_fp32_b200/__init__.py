@@ -83,6 +83,7 @@ _SIGS = {
     "moe_layer_forward_fp8": ([_SP, _vp, _WP, _FP, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
                               ctypes.c_int),
     "moe_set_variant": ([ctypes.c_int], ctypes.c_int),
+    "moe_workspace_set_variant": ([_vp, _sz, ctypes.c_int], ctypes.c_int),
     "moe_compact_workspace_bytes": ([_SP], _sz),
     "moe_zero_channel_count": ([_SP, _vp, ctypes.POINTER(ctypes.c_int32), _vp, _sz, _vp], ctypes.c_int),
     "moe_compact_zero_channels": ([_SP, _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
@@ -272,7 +273,14 @@ def moe_layer_forward_fp8(shape, x, weights, experts, out, ws, topk_ids=None, to
 
 
 def moe_set_variant(variant: int) -> None:
+    """Process-wide default variant (used by workspaces without a choice of their own)."""
     _check(_lib.moe_set_variant(int(variant)), "moe_set_variant")
+
+
+def moe_workspace_set_variant(ws, variant: int) -> None:
+    """Variant for the calls made with workspace `ws`."""
+    _check(_lib.moe_workspace_set_variant(_ptr(ws), _nbytes(ws), int(variant)),
+           "moe_workspace_set_variant")
 
 
 def moe_device_status(ws, stream=None):
@@ -305,13 +313,17 @@ def moe_launch_count() -> int:
 
 # --------------------------------------------------------------------------- conveniences
 
-def alloc_workspace(shape: moe_shape, device="cuda", host_staging: bool = False, stream=None):
-    """A uint8 device tensor sized for `shape`, with its status word cleared."""
+def alloc_workspace(shape: moe_shape, device="cuda", host_staging: bool = False, stream=None,
+                    variant: Optional[int] = None):
+    """A uint8 device tensor sized for `shape`, with its status word cleared (and its own
+    grouped-GEMM variant, if `variant` is given)."""
     import torch
 
     n = moe_workspace_bytes(shape) + (moe_host_staging_bytes(shape) if host_staging else 0)
     ws = torch.empty(n, dtype=torch.uint8, device=device)
     moe_workspace_init(ws, stream)
+    if variant is not None:
+        moe_workspace_set_variant(ws, variant)
     return ws
 
 

@@ -47,7 +47,6 @@ zero_channel_mask_kernel(const uint16_t* __restrict__ w_gate_up, int E, int I, i
 
 // One block per expert: src[e][j] = the j-th live channel (j < count), -1 for j in
 // [count, Ic); count[e] = number of live channels. A count above Ic is flagged.
-constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads)
 zero_channel_scan_kernel(const uint8_t* __restrict__ live, int E, int I, int Ic,
                          int32_t* __restrict__ src, int32_t* __restrict__ count,

@@ -77,4 +77,37 @@ __device__ __forceinline__ void set_flag(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
+constexpr int kScanThreads = 1024;
+
+// Block-wide exclusive scan of one value per thread; blockDim.x must be kScanThreads (32
+// warps). Returns this thread's exclusive prefix; *total receives the block's sum.
+__device__ inline int block_exclusive_scan(int v, int* smem_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) smem_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int s = smem_warp[lane];
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += n;
+    }
+    smem_warp[lane] = si - s;  // exclusive warp prefix
+    if (lane == 31) smem_warp[32] = si;
+  }
+  __syncthreads();
+  const int r = smem_warp[warp] + incl - v;
+  *total = smem_warp[32];
+  __syncthreads();
+  return r;
+}
+
+
 }  // namespace moe

@@ -4,6 +4,7 @@
 // Dispatch R tokens -> Grouped expert GEMMs -> Weighted combine + gated shared expert").
 #include <atomic>
 #include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "moe_internal.h"
@@ -51,7 +52,10 @@ Layout layout(const moe_shape& s) {
 namespace {
 
 std::atomic<uint64_t> g_launches{0};
-std::atomic<int> g_variant{MOE_VARIANT_AUTO};
+std::atomic<int> g_variant{MOE_VARIANT_AUTO};  // process-wide default
+// per-workspace choices (moe_workspace_set_variant), keyed by the workspace's address
+std::mutex g_ws_variant_mu;
+std::unordered_map<const void*, int> g_ws_variant;
 std::mutex g_prof_mu;
 bool g_prof_on = false;
 struct ProfRec {
@@ -134,6 +138,13 @@ moe_status check_expert_weights(const moe_weights* w) {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+int sm_count_host() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 #define MOE_TRY(expr)                     \
   do {                                    \
     moe_status _st = (expr);              \
@@ -141,11 +152,21 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
   } while (0)
 #define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
 
+// The variant for calls on workspace `ws`: its own choice if one was set, else the
+// process-wide default.
+int variant_of(const void* ws) {
+  {
+    std::lock_guard<std::mutex> lk(g_ws_variant_mu);
+    auto it = g_ws_variant.find(ws);
+    if (it != g_ws_variant.end()) return it->second;
+  }
+  return g_variant.load();
+}
+
 // Tensor-core variant for this shape? AUTO takes it wherever the shape allows: on B200 it
 // streams the activated experts' weights faster than the CUDA-core kernels even at
 // decode sizes (a 16-token MMA tile costs nothing next to the weight bytes).
-bool use_tc(const moe_shape& s) {
-  const int v = g_variant.load();
+bool use_tc(const moe_shape& s, int v) {
   if (v == MOE_VARIANT_STREAM) return false;
   return tc_supported(s);
 }
@@ -155,26 +176,23 @@ bool use_tc(const moe_shape& s) {
 // 2.4T-shaped prefill 8001 / 6941); the gate|up GEMM only once the token tiles are wide
 // (decode 384 / 393; 2.4T-shaped prefill 6986 / 6921; Flash-Next prefill 780 / 709), which
 // AUTO takes as an average of at least 16 routed rows per expert.
-bool use_tc2_gate_up(const moe_shape& s) {
-  const int v = g_variant.load();
+bool use_tc2_gate_up(const moe_shape& s, int v) {
   if (v == MOE_VARIANT_TC2) return true;
   return v == MOE_VARIANT_AUTO && (int64_t)s.T * s.k >= 16 * (int64_t)s.E;
 }
 
-bool use_tc2_down(const moe_shape& s) {
-  const int v = g_variant.load();
-  return v == MOE_VARIANT_TC2 || v == MOE_VARIANT_AUTO;
-}
+bool use_tc2_down(int v) { return v == MOE_VARIANT_TC2 || v == MOE_VARIANT_AUTO; }
 
 // Stage 4 on the plan in the workspace: fused (out != NULL) or per-row y / y_shared.
 moe_status run_grouped(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                        const int32_t* sorted_token, const float* sorted_w, const float* sgate,
                        const moe_weights& w, float* y, float* y_shared, float* out,
                        cudaStream_t st) {
-  if (use_tc(s)) {
-    if (use_tc2_gate_up(s)) MOE_CUDA(launch_tc2_gate_up(s, L, ws, x, sorted_token, w, st));
+  const int v = variant_of(ws);
+  if (use_tc(s, v)) {
+    if (use_tc2_gate_up(s, v)) MOE_CUDA(launch_tc2_gate_up(s, L, ws, x, sorted_token, w, st));
     else MOE_CUDA(launch_tc_gate_up(s, L, ws, x, sorted_token, w, st));
-    if (use_tc2_down(s))
+    if (use_tc2_down(v))
       MOE_CUDA(launch_tc2_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));
     else
       MOE_CUDA(launch_tc_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));
@@ -202,6 +220,10 @@ size_t moe_host_staging_bytes(const moe_shape* shape) {
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (!aligned16(ws) || ws_bytes < 256) return MOE_ERR_INVALID_ARG;
+  {
+    std::lock_guard<std::mutex> lk(g_ws_variant_mu);
+    g_ws_variant.erase(ws);
+  }
   MOE_CUDA(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream));
   return MOE_OK;
 }
@@ -250,19 +272,29 @@ moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const int32
                               const int32_t* offsets, const moe_weights* weights, float* y,
                               float* y_shared, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(check_shape(shape));
-  const moe_shape& s = *shape;
-  MOE_TRY(check_expert_weights(weights));
+  if (!weights) return MOE_ERR_INVALID_ARG;
+  // both shared-expert matrices NULL: routed experts only (y_shared is not written)
+  const bool shared = weights->ws_gate_up || weights->ws_down;
+  moe_weights wv = *weights;
+  moe_shape s = *shape;
+  if (!shared) {
+    // no tile reads the shared expert's matrices; its tensor maps still need a valid base
+    wv.ws_gate_up = wv.w_gate_up;
+    wv.ws_down = wv.w_down;
+    s.Is = s.I;  // the workspace layout for Is = I is no larger than the caller's
+  }
+  MOE_TRY(check_expert_weights(&wv));
   if (!aligned16(x) || !aligned16(sorted_token) || !aligned16(offsets) || !aligned16(y) ||
-      !aligned16(y_shared))
+      (shared && !aligned16(y_shared)))
     return MOE_ERR_INVALID_ARG;
-  MOE_TRY(check_ws(s, ws, ws_bytes));
+  MOE_TRY(check_ws(*shape, ws, ws_bytes));
   if (s.T == 0) return MOE_OK;
   const Layout L = layout(s);
   char* w = static_cast<char*>(ws);
   cudaStream_t st = (cudaStream_t)stream;
-  MOE_CUDA(launch_plan_from_offsets(s, L, w, offsets, st));
-  return run_grouped(s, L, w, static_cast<const uint16_t*>(x), sorted_token, nullptr, nullptr,
-                     *weights, y, y_shared, nullptr, st);
+  MOE_CUDA(launch_plan_from_offsets(s, L, w, offsets, shared ? s.T : 0, st));
+  return run_grouped(s, L, w, static_cast<const uint16_t*>(x), sorted_token, nullptr, nullptr, wv,
+                     y, shared ? y_shared : nullptr, nullptr, st);
 }
 
 moe_status moe_unpermute_combine(const moe_shape* shape, const float* y, const float* y_shared,
@@ -446,11 +478,59 @@ moe_status moe_layer_forward_fp8(const moe_shape* shape, const void* x, const mo
   return MOE_OK;
 }
 
-moe_status moe_set_variant(moe_variant variant) {
-  if (variant != MOE_VARIANT_AUTO && variant != MOE_VARIANT_STREAM && variant != MOE_VARIANT_TC &&
-      variant != MOE_VARIANT_TC2)
+static bool valid_variant(moe_variant v) {
+  return v == MOE_VARIANT_AUTO || v == MOE_VARIANT_STREAM || v == MOE_VARIANT_TC ||
+         v == MOE_VARIANT_TC2;
+}
+
+moe_status moe_gather_rows(int64_t rows, int32_t H, const void* x, int64_t n_src,
+                           const int32_t* index, void* out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  if (rows < 0 || n_src < 0 || H <= 0 || H % 8) return MOE_ERR_INVALID_ARG;
+  if (ws && (!aligned16(ws) || ws_bytes < 256)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!aligned16(x) || !aligned16(index) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(launch_gather_rows_bf16(static_cast<const uint16_t*>(x), index, rows, n_src, H,
+                                   static_cast<uint16_t*>(out), static_cast<uint32_t*>(ws),
+                                   sm_count_host(), (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+moe_status moe_scatter_rows(int64_t rows, int32_t H, const float* y, int64_t n_dst,
+                            const int32_t* index, float* out, void* ws, size_t ws_bytes,
+                            void* stream) {
+  if (rows < 0 || n_dst < 0 || H <= 0 || H % 4) return MOE_ERR_INVALID_ARG;
+  if (ws && (!aligned16(ws) || ws_bytes < 256)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!aligned16(y) || !aligned16(index) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(launch_scatter_rows_f32(y, index, rows, n_dst, H, out, static_cast<uint32_t*>(ws),
+                                   sm_count_host(), (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+moe_status moe_ep_regroup(int32_t G, int32_t E_local, const int32_t* recv_counts,
+                          int64_t capacity, int32_t* offsets, int32_t* src_index, void* ws,
+                          size_t ws_bytes, void* stream) {
+  if (G <= 0 || E_local <= 0 || capacity < 0) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)G * E_local > kMaxE || capacity >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(recv_counts) || !aligned16(offsets) || (capacity > 0 && !aligned16(src_index)))
     return MOE_ERR_INVALID_ARG;
+  if (ws && (!aligned16(ws) || ws_bytes < 256)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(launch_ep_regroup(recv_counts, G, E_local, capacity, offsets, src_index,
+                             static_cast<uint32_t*>(ws), (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+moe_status moe_set_variant(moe_variant variant) {
+  if (!valid_variant(variant)) return MOE_ERR_INVALID_ARG;
   g_variant.store((int)variant);
+  return MOE_OK;
+}
+
+moe_status moe_workspace_set_variant(void* ws, size_t ws_bytes, moe_variant variant) {
+  if (!aligned16(ws) || ws_bytes < 256 || !valid_variant(variant)) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_ws_variant_mu);
+  g_ws_variant[ws] = (int)variant;
   return MOE_OK;
 }
 

@@ -111,8 +111,19 @@ cudaError_t launch_router_topk(const moe_shape& s, const float* logits, const fl
 cudaError_t launch_permute(const moe_shape& s, const Layout& L, char* ws, const int32_t* ids,
                            const float* topk_w, int32_t* offsets, int32_t* sorted_token,
                            float* sorted_w, int32_t* assign_row, cudaStream_t st);
+// Plan from caller-supplied offsets; shared_rows = T with the shared expert, 0 without.
 cudaError_t launch_plan_from_offsets(const moe_shape& s, const Layout& L, char* ws,
-                                     const int32_t* offsets, cudaStream_t st);
+                                     const int32_t* offsets, int shared_rows, cudaStream_t st);
+// Expert-parallel row movement (ep.cu).
+cudaError_t launch_gather_rows_bf16(const uint16_t* x, const int32_t* index, int64_t rows,
+                                    int64_t n_src, int H, uint16_t* out, uint32_t* status,
+                                    int sms, cudaStream_t st);
+cudaError_t launch_scatter_rows_f32(const float* y, const int32_t* index, int64_t rows,
+                                    int64_t n_dst, int H, float* out, uint32_t* status, int sms,
+                                    cudaStream_t st);
+cudaError_t launch_ep_regroup(const int32_t* counts, int G, int El, int64_t capacity,
+                              int32_t* offsets, int32_t* src_index, uint32_t* status,
+                              cudaStream_t st);
 cudaError_t launch_stream_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                                   const int32_t* sorted_token, const moe_weights& w,
                                   cudaStream_t st);

@@ -23,8 +23,6 @@
 namespace moe {
 namespace {
 
-constexpr int kScanThreads = 1024;
-
 __global__ void __launch_bounds__(kPermBlock)
 dispatch_mask_kernel(const int32_t* __restrict__ ids, int T, int E, int k,
                      uint32_t* __restrict__ blk_mask, int32_t* __restrict__ blk_count,
@@ -54,35 +52,6 @@ dispatch_mask_kernel(const int32_t* __restrict__ ids, int T, int E, int k,
     for (int w = 0; w < 8; ++w) c += __popc(mask[e * 8 + w]);
     blk_count[(size_t)b * E + e] = c;
   }
-}
-
-// Block-wide exclusive scan of one value per thread (blockDim.x == kScanThreads).
-__device__ int block_exclusive_scan(int v, int* smem_warp, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  if (lane == 31) smem_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int s = smem_warp[lane];
-    int si = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, si, o);
-      if (lane >= o) si += n;
-    }
-    smem_warp[lane] = si - s;  // exclusive warp prefix
-    if (lane == 31) smem_warp[32] = si;
-  }
-  __syncthreads();
-  const int r = smem_warp[warp] + incl - v;
-  *total = smem_warp[32];
-  __syncthreads();
-  return r;
 }
 
 // Group sizes n_g (g < E routed, g == E shared = T) -> plan. Called by all threads of a
@@ -254,7 +223,8 @@ dispatch_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__
 // T*k rows starting at 0 are flagged and give an empty plan (no GEMM work).
 __global__ void __launch_bounds__(kScanThreads)
 plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int T, int E, int k, int H, int I,
-                         int Is, int* __restrict__ plan_base, uint32_t* __restrict__ status) {
+                         int Is, int shared_rows, int* __restrict__ plan_base,
+                         uint32_t* __restrict__ status) {
   __shared__ int smem[33];
   __shared__ int n_of[kMaxE + 1];
   __shared__ int bad;
@@ -265,7 +235,7 @@ plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int T, int E, int 
     if (n < 0) bad = 1;
     n_of[g] = n;
   }
-  if (threadIdx.x == 0) n_of[E] = T;
+  if (threadIdx.x == 0) n_of[E] = shared_rows;
   __syncthreads();
   if (bad) {
     for (int g = threadIdx.x; g <= E; g += blockDim.x) n_of[g] = 0;
@@ -305,10 +275,10 @@ cudaError_t launch_permute(const moe_shape& s, const Layout& L, char* ws, const 
 }
 
 cudaError_t launch_plan_from_offsets(const moe_shape& s, const Layout& L, char* ws,
-                                     const int32_t* offsets, cudaStream_t st) {
+                                     const int32_t* offsets, int shared_rows, cudaStream_t st) {
   LaunchScope scope(MOE_K_PERMUTE, st);
   plan_from_offsets_kernel<<<1, kScanThreads, 0, st>>>(
-      offsets, s.T, s.E, s.k, s.H, s.I, s.Is, reinterpret_cast<int*>(ws + L.plan),
+      offsets, s.T, s.E, s.k, s.H, s.I, s.Is, shared_rows, reinterpret_cast<int*>(ws + L.plan),
       reinterpret_cast<uint32_t*>(ws + L.status));
   return cudaGetLastError();
 }
@@ -320,7 +290,9 @@ cudaError_t launch_plan_from_offsets(const moe_shape& s, const Layout& L, char* 
 // GEMM plan -- lives in one file-scope device array that every GPU loading this library
 // holds until the process exits. In host code `g_noalloc_scratch` is only a host-side
 // stand-in for the symbol; its device address is looked up with cudaGetSymbolAddress,
-// once per device, with that device current (the first call on a device does it).
+// once per device, with that device current (the first call on a device does it). The
+// address is kept for the life of the process, so the entry point must not be used after a
+// cudaDeviceReset (or any teardown of the device's primary context) in the same process.
 
 namespace {
 
@@ -402,6 +374,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t*
   uint32_t* blk_mask = reinterpret_cast<uint32_t*>(ws + L.blk_mask);
   int32_t* blk_base = reinterpret_cast<int32_t*>(ws + L.blk_base);
   const size_t smem = (size_t)s.E * 8 * sizeof(uint32_t);
+  LaunchScope scope(MOE_K_PERMUTE, st, 3);
   dispatch_mask_kernel<<<L.nblk, kPermBlock, smem, st>>>(topk_ids, s.T, s.E, s.k, blk_mask,
                                                         blk_base, status);
   dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(blk_base, L.nblk, s.T, s.E, s.k, s.H, s.I,

@@ -323,7 +323,6 @@ int router_slices(const moe_shape& s) { return s.T < kTcRouterMinTokens ? kSplit
 cudaError_t launch_router_logits(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                                  const float* wr, float* logits, cudaStream_t st) {
   const int nslices = router_slices(s);
-  const bool tc_logits = nslices == 1 && tc_router_supported(s);
   if (nslices == 1 && tc_router_supported(s)) return launch_tc_router(s, L, ws, x, wr, logits, st);
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;

@@ -1,5 +1,5 @@
 // sm100_ptx.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features the
-// tensor-core kernels use: mbarriers, TMA tensor loads (tiled and 4-row gather),
+// tensor-core kernels use: mbarriers, tiled TMA tensor loads,
 // tcgen05 tensor-memory allocation, MMA issue/commit and TMEM loads. Written from the
 // public PTX ISA; every wait built on these is bounded by the caller.
 #pragma once
@@ -77,18 +77,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_
       : "memory");
 }
 
-// Four rows r0..r3 (outer coordinates) of the column box starting at `col`, written as
-// four consecutive box rows in shared memory (tensor map box: one row high).
-__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, uint64_t* bar, int col,
-                                            int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1),
-      "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -112,19 +100,6 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulate (kind::f16).
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n"
-      " .reg .pred p;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
-      "}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // Back-to-back MMAs over consecutive 16-wide K steps, issued from one asm block so that no
@@ -219,10 +194,6 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(const void* p) {
          (layout << 61);
 }
 
-__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
-  return smem_desc_kmajor<128>(p);
-}
-
 // Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
@@ -302,19 +273,6 @@ __device__ __forceinline__ void tmem_relinquish_pair() {
 __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
-}
-
-// D (+)= A * B^T over the pair (M = 256), bf16 inputs, fp32 accumulate; leader CTA only.
-__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                               uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n"
-      " .reg .pred p;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n"
-      "}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // Arrive once on the mbarrier at the same shared offset in every CTA of `cta_mask` when all

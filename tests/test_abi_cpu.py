@@ -106,6 +106,17 @@ def test_variant_setter():
         moe.moe_set_variant(v)
 
 
+def test_workspace_variant_setter_checks_its_arguments():
+    # host-side bookkeeping only: no GPU is touched, so fake aligned addresses serve
+    L = moe.lib()
+    assert L.moe_workspace_set_variant(4096, 1 << 20, 7) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_workspace_set_variant(4100, 1 << 20, moe.MOE_VARIANT_TC) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_workspace_set_variant(None, 1 << 20, moe.MOE_VARIANT_TC) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_workspace_set_variant(4096, 128, moe.MOE_VARIANT_TC) == moe.MOE_ERR_INVALID_ARG
+    for v in (moe.MOE_VARIANT_STREAM, moe.MOE_VARIANT_TC, moe.MOE_VARIANT_TC2, moe.MOE_VARIANT_AUTO):
+        assert L.moe_workspace_set_variant(4096, 1 << 20, v) == moe.MOE_OK
+
+
 def test_profile_collect_empty():
     moe.moe_profile_enable(True)
     moe.moe_profile_enable(False)

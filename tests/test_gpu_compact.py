@@ -29,12 +29,6 @@ def _u16(t):
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-@pytest.fixture(autouse=True)
-def _variant_reset():
-    yield
-    moe.moe_set_variant(moe.MOE_VARIANT_AUTO)
-
-
 def _edit_rows(gu_dev, gu_host, I):
     """Extra dead channels beyond the generator's: gate-only, up-only, -0.0 rows, and a
     channel kept alive by one nonzero value. The same edits go to both copies."""
@@ -104,10 +98,8 @@ def _check_rows(cfg, host, out, ids, rows):
 def _forward_compacted(cfg, dev, variant=None):
     s = moe.shape_of(cfg)
     wc, I_c = moe.compact_zero_channels(s, dev)
-    if variant is not None:
-        moe.moe_set_variant(variant)
     sc = moe.shape_of(cfg.replace(I=I_c))
-    ws = moe.alloc_workspace(sc)
+    ws = moe.alloc_workspace(sc, variant=variant)
     out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
     ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
     moe.moe_layer_forward(sc, dev["x"], wc, out, ws, topk_ids=ids)

@@ -1,0 +1,275 @@
+"""GPU parity at the full prefill sizes, through the C ABI, against the fp64 oracle.
+
+The workloads: Flash-Next-shaped prefill (T=8192, hidden 2560), 2.4T-shaped prefill
+(T=8192, hidden 8192) and the skewed 2.4T-shaped layer (T=16384, Zipf router bias, 71 %
+zero gate/up channels), each run in full on the GPU. The oracle evaluates chosen parts of
+the same run, so the checks aim at the tiles where a fault would hide:
+
+* the staged entry points (moe_permute -> moe_grouped_swiglu -> moe_unpermute_combine) on
+  the oracle's routing: per-assignment outputs y for every packed row of the first and the
+  last (ragged) tiles of the hottest expert, the coldest expert and others; y_shared for
+  the shared expert's first and last tiles; the combine on the GPU's own y and y_shared
+  (exact inputs), and the combined output against the oracle's layer;
+* the fused layer forward in the launch configuration the benchmark times: at least 128
+  tokens, including every token of the hottest expert's last partial tile and of the
+  shared expert's last tile.
+
+Tiles follow the kernels' plan: a group of n packed rows is split into ceil(n / max)
+near-equal chunks of a multiple of 16 rows (max 256 for gate|up, 128 for down).
+Tolerance: max |gpu - ref| <= 1e-2 RMS(ref), mean relative error <= 2e-3; routing id
+sets exact except near-ties (10th/11th fp64 logit gap < 1e-5).
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU, skipped there
+    pytestmark = pytest.mark.skip(reason="needs a CUDA device")
+
+import oracle  # noqa: E402
+import sparse_moe_expert_fp32_b200 as moe  # noqa: E402
+import synth  # noqa: E402
+from parity_util import assert_layer_close, id_sets_match  # noqa: E402
+
+VARIANTS = {"stream": moe.MOE_VARIANT_STREAM, "tc": moe.MOE_VARIANT_TC,
+            "tc2": moe.MOE_VARIANT_TC2, "auto": moe.MOE_VARIANT_AUTO}
+FULL = ["flash_prefill", "t24_prefill", "t24_skewed"]
+GATE_UP_TILE, DOWN_TILE = 256, 128
+
+
+def _chunks(n, max_rows):
+    """[(start, rows)] of the kernels' split of a group of n rows."""
+    nch = -(-n // max_rows)
+    cs = ((-(-n // nch)) + 15) & ~15
+    return [(c * cs, min(cs, n - c * cs)) for c in range(nch)]
+
+
+def _last_tile_rows(n):
+    """Row range [a, n) covering the last gate|up tile and the last down tile of a group."""
+    a = min(_chunks(n, GATE_UP_TILE)[-1][0], _chunks(n, DOWN_TILE)[-1][0])
+    return a, n
+
+
+# ----------------------------------------------------------------------------- shared state
+# One workload's inputs and oracle results at a time (host and device), reused by every
+# variant of that workload; the tests run workload by workload.
+
+_CACHE = {}
+
+
+def _state(name):
+    if _CACHE.get("name") != name:
+        _CACHE.clear()
+        torch.cuda.empty_cache()
+        cfg = synth.CONFIGS[name]
+        host = synth.host_inputs(cfg, seed=0)
+        logits = oracle.router_logits(host.x, host.w_router, host.router_bias)
+        ids, gap = oracle.topk_select(logits, cfg.k)
+        offsets, sorted_token, assign_row, _ = oracle.permute(ids, cfg.E)
+        _CACHE.update(name=name, cfg=cfg, host=host, logits=logits, ids=ids, gap=gap,
+                      offsets=offsets, sorted_token=sorted_token, assign_row=assign_row,
+                      weights=oracle.routing_weights(logits, ids),
+                      sgate=oracle.shared_gate(host.x, host.w_shared_gate),
+                      dev=synth.device_inputs(cfg, seed=0))
+    return _CACHE
+
+
+def _hottest(st):
+    counts = np.diff(st["offsets"])
+    return int(np.argmax(counts)), counts
+
+
+def _chosen_experts(st):
+    """Hottest, coldest non-empty, the most ragged multi-tile group, two seeded others."""
+    hot, counts = _hottest(st)
+    nz = np.nonzero(counts)[0]
+    cold = int(nz[np.argmin(counts[nz])])
+    multi = [int(e) for e in nz if counts[e] > DOWN_TILE]
+    ragged = max(multi, key=lambda e: (counts[e] % 16 != 0, counts[e] % 128), default=hot)
+    rng = np.random.default_rng(5)
+    others = [int(e) for e in rng.choice(nz, 2, replace=False)]
+    return sorted(set([hot, cold, ragged] + others))
+
+
+def _staged_expect(st):
+    """Oracle y rows (first 64 and last tiles of chosen experts), y_shared rows (first and
+    last shared tiles) and the layer on a few tokens; computed once per workload."""
+    if "staged" in st:
+        return st["staged"]
+    cfg, host = st["cfg"], st["host"]
+    x64 = oracle.bf16_to_f64(host.x)
+    rows, yref = [], []
+    for e in _chosen_experts(st):
+        a0, a1 = int(st["offsets"][e]), int(st["offsets"][e + 1])
+        n = a1 - a0
+        lo, hi = _last_tile_rows(n)
+        r = sorted(set(range(min(n, 64))) | set(range(lo, hi)))
+        p = [a0 + i for i in r]
+        toks = st["sorted_token"][p]
+        yref.append(oracle.swiglu_expert(x64[toks], host.gate_up(e), host.down(e)))
+        rows.extend(p)
+    T = cfg.T
+    sh_rows = sorted(set(range(GATE_UP_TILE)) | set(range(T - GATE_UP_TILE, T)))
+    ysh = oracle.swiglu_expert(x64[sh_rows], host.ws_gate_up, host.ws_down)
+    rng = np.random.default_rng(11)
+    layer_rows = sorted(set([0, T - 1] + rng.choice(T, 10, replace=False).tolist()))
+    ref = oracle.forward_inputs(host, rows=layer_rows)
+    st["staged"] = dict(rows=np.array(rows), y=np.concatenate(yref), sh_rows=np.array(sh_rows),
+                        y_shared=ysh, layer_rows=layer_rows, out=ref["out"])
+    return st["staged"]
+
+
+def _dev(a, dtype):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=dtype)).cuda()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,variant", [(n, v) for n in FULL for v in ("tc", "tc2", "auto")])
+def test_staged_entry_points_full_size(name, variant):
+    st = _state(name)
+    cfg, dev = st["cfg"], st["dev"]
+    exp = _staged_expect(st)
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s, variant=VARIANTS[variant])
+    R, T, H = cfg.R, cfg.T, cfg.H
+    off = torch.empty(cfg.E + 1, dtype=torch.int32, device="cuda")
+    stok = torch.empty(R, dtype=torch.int32, device="cuda")
+    ar = torch.empty(R, dtype=torch.int32, device="cuda")
+    moe.moe_permute(s, _dev(st["ids"], np.int32), off, stok, ar, ws)
+    assert np.array_equal(off.cpu().numpy(), st["offsets"])
+    assert np.array_equal(stok.cpu().numpy(), st["sorted_token"])
+    y = torch.full((R, H), float("nan"), dtype=torch.float32, device="cuda")
+    ys = torch.full((T, H), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_grouped_swiglu(s, dev["x"], stok, off, dev, y, ys, ws)
+    w = _dev(st["weights"], np.float32)
+    sg = _dev(st["sgate"], np.float32)
+    out = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    moe.moe_unpermute_combine(s, y, ys, ar, w, sg, out)
+    status, flags = moe.moe_device_status(ws)
+    assert status == moe.MOE_OK, (status, flags)
+    # every packed row and shared row was written (no NaN left from the fill)
+    assert not torch.isnan(y).any().item() and not torch.isnan(ys).any().item()
+
+    gy = y[torch.from_numpy(exp["rows"]).cuda()].cpu().numpy()
+    assert_layer_close(gy, exp["y"], f"{name} {variant} y (chosen experts' first and last tiles)")
+    gys = ys[torch.from_numpy(exp["sh_rows"]).cuda()].cpu().numpy()
+    assert_layer_close(gys, exp["y_shared"], f"{name} {variant} y_shared (first and last tiles)")
+
+    # combine on the GPU's own y, y_shared: the stated fixed-order sum, fp32 vs fp64
+    rng = np.random.default_rng(3)
+    toks = sorted(set([0, T - 1] + rng.choice(T, 254, replace=False).tolist()))
+    arow = st["assign_row"][toks]
+    yk = y[torch.from_numpy(arow.reshape(-1)).cuda()].cpu().numpy().reshape(len(toks), cfg.k, H)
+    ysk = ys[torch.tensor(toks).cuda()].cpu().numpy()
+    ref_c = oracle.combine(yk.reshape(-1, H), ysk, np.arange(len(toks) * cfg.k).reshape(len(toks), cfg.k),
+                           st["weights"][toks], st["sgate"][toks])
+    assert np.allclose(out[torch.tensor(toks).cuda()].cpu().numpy(), ref_c, rtol=1e-5, atol=1e-5)
+
+    # combined output against the oracle's layer on the same routing
+    lr = exp["layer_rows"]
+    assert_layer_close(out[torch.tensor(lr).cuda()].cpu().numpy(), exp["out"], f"{name} {variant} out")
+    del y, ys, out, ws
+    torch.cuda.empty_cache()
+
+
+def _layer_rows(st):
+    """>= 128 tokens: every token of the hottest expert's last tiles, the shared expert's
+    last down tile and every 8th token of the rest of its last gate|up tile, the first and
+    last tokens, and seeded others."""
+    cfg = st["cfg"]
+    T = cfg.T
+    hot, counts = _hottest(st)
+    a0 = int(st["offsets"][hot])
+    lo, hi = _last_tile_rows(int(counts[hot]))
+    hot_toks = st["sorted_token"][a0 + lo:a0 + hi].tolist()
+    shared = list(range(T - DOWN_TILE, T)) + list(range(T - GATE_UP_TILE, T - DOWN_TILE, 8))
+    rng = np.random.default_rng(123)
+    rows = set(hot_toks) | set(shared) | {0} | set(rng.choice(T, 32, replace=False).tolist())
+    rows = sorted(rows)
+    assert len(rows) >= 128
+    return rows, hot, len(hot_toks)
+
+
+def _layer_expect(st):
+    if "layer" not in st:
+        rows, hot, nhot = _layer_rows(st)
+        ref = oracle.forward_inputs(st["host"], rows=rows)
+        st["layer"] = dict(rows=rows, ref=ref, hot=hot, nhot=nhot)
+    return st["layer"]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,variant", [(n, v) for n in FULL for v in ("auto", "tc2", "tc", "stream")])
+def test_layer_forward_full_size_sampled(name, variant):
+    st = _state(name)
+    cfg, dev = st["cfg"], st["dev"]
+    exp = _layer_expect(st)
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s, variant=VARIANTS[variant])
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    moe.moe_layer_forward(s, dev["x"], dev, out, ws, topk_ids=ids)
+    status, flags = moe.moe_device_status(ws)
+    assert status == moe.MOE_OK, (status, flags)
+    rows = exp["rows"]
+    sel = torch.tensor(rows).cuda()
+    gout, gids = out[sel].cpu().numpy(), ids[sel].cpu().numpy()
+    ref = exp["ref"]
+    differ = id_sets_match(gids, ref["ids"], ref["gap"], ref["logits"])
+    keep = [i for i in range(len(rows)) if i not in set(differ)]
+    stats = assert_layer_close(gout[keep], ref["out"][keep], f"{name} {variant}")
+    print(name, variant, len(rows), "tokens (hottest expert", exp["hot"], "last tiles:", exp["nhot"],
+          "tokens)", stats, "near-ties", len(differ))
+    del out, ws
+    torch.cuda.empty_cache()
+
+
+def test_tile_split_matches_the_kernels_plan():
+    # the split the tests aim at: near-equal chunks, multiples of 16, covering all rows
+    for n in (1, 15, 16, 17, 128, 129, 210, 256, 257, 1000, 8000):
+        for m in (GATE_UP_TILE, DOWN_TILE):
+            ch = _chunks(n, m)
+            assert sum(r for _, r in ch) == n and all(r > 0 for _, r in ch)
+            assert all(a % 16 == 0 for a, _ in ch) and max(r for _, r in ch) <= m
+    assert _last_tile_rows(210) == (128, 210) and _last_tile_rows(100) == (0, 100)
+
+
+# ----------------------------------------------------------------------------- router ties
+
+@pytest.mark.gpu
+def test_tensor_core_router_ties_go_to_lower_index():
+    """T >= 512 takes the tensor-core router (exact bf16 split of the fp32 router matrix,
+    then exact fp32 recomputation near the decision). Experts e, e+170 and e+340 share one
+    router row, so every token's top-10 holds three whole triples and one member of a
+    fourth: the tie straddles the 10th/11th place on every token, and the lower index
+    must win each time."""
+    cfg = synth.CONFIGS["flash_decode"].replace(name="tc_router_ties", T=640)
+    dev = synth.device_inputs(cfg, seed=4)
+    wr = dev["w_router"]
+    for e in range(170):
+        wr[e + 170] = wr[e]
+        wr[e + 340] = wr[e]
+    s = moe.shape_of(cfg)
+    ws = moe.alloc_workspace(s)
+    ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device="cuda")
+    sg = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
+    gap = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
+    moe.moe_router_topk(s, dev["x"], dev, ids, tw, sg, gap, ws)
+    assert moe.moe_device_status(ws)[0] == moe.MOE_OK
+    x = dev["x"].view(torch.int16).cpu().numpy().view(np.uint16)
+    logits = oracle.router_logits(x, wr.cpu().numpy())
+    rids, rgap = oracle.topk_select(logits, cfg.k)
+    gids = ids.cpu().numpy()
+    straddle = 0
+    for t in range(cfg.T):
+        assert set(gids[t].tolist()) == set(rids[t].tolist()), (t, sorted(gids[t]), sorted(rids[t]))
+        base = {int(e) % 170 for e in gids[t] if e < 510}
+        for b in base:
+            members = [m for m in (b, b + 170, b + 340) if m in set(gids[t].tolist())]
+            # a partly chosen triple keeps its lowest indices
+            assert members == [b, b + 170, b + 340][:len(members)], (t, b, members)
+        straddle += rgap[t] == 0.0
+    assert straddle >= cfg.T // 2  # the tie sits at the decision on most tokens
+    assert np.allclose(tw.cpu().numpy().sum(axis=1), 1.0, atol=1e-5)

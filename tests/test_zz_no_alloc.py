@@ -28,7 +28,9 @@ def test_noalloc_dispatch_equals_workspace_dispatch_two_calls():
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    cases = [(1000, 512, 10, 11), (300, 64, 8, 12)]  # two calls in a row, different routing
+    # calls in a row with different routing; the decode-size batches (T <= 256) compare the
+    # no-allocation path against moe_permute's one-kernel small-batch dispatch
+    cases = [(1000, 512, 10, 11), (300, 64, 8, 12), (64, 512, 10, 13), (1, 16, 4, 14)]
     for T, E, k, seed in cases:
         s = moe.make_shape(T, 256, E, k, 128, 128)
         ids = torch.from_numpy(_ids(T, E, k, seed)).cuda()
@@ -55,3 +57,35 @@ def test_noalloc_refuses_shapes_beyond_its_scratch():
     assert st == moe.MOE_ERR_UNSUPPORTED
     s_ok = moe.make_shape(0, 256, 512, 10, 128, 128)  # empty batch: valid, no work
     assert moe.lib().moe_permute_noalloc(ctypes.byref(s_ok), 16, 16, 16, 16, None) == moe.MOE_OK
+
+
+@pytest.mark.gpu
+def test_noalloc_skips_an_out_of_range_id_like_moe_permute():
+    """One assignment names expert E: it is skipped, offsets[E] falls one short of T*k, and
+    every other output equals moe_permute's on the same ids."""
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    T, E, k = 300, 64, 8
+    ids_np = _ids(T, E, k, 15)
+    ids_np[123, 4] = E
+    s = moe.make_shape(T, 256, E, k, 128, 128)
+    ids = torch.from_numpy(ids_np).cuda()
+    ref_off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    ref_st = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    ref_ar = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    ws = moe.alloc_workspace(s)
+    moe.moe_permute(s, ids, ref_off, ref_st, ref_ar, ws)
+    assert moe.moe_device_status(ws)[0] == moe.MOE_ERR_DEVICE_BOUNDS
+    off = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    st = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    ar = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    moe.moe_permute_noalloc(s, ids, off, st, ar)
+    torch.cuda.synchronize()
+    assert int(off[-1]) == T * k - 1
+    assert torch.equal(off, ref_off)
+    n = T * k - 1
+    assert torch.equal(st[:n], ref_st[:n])
+    keep = torch.ones(T * k, dtype=torch.bool, device="cuda")
+    keep[123 * k + 4] = False
+    assert torch.equal(ar[keep], ref_ar[keep])
