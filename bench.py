@@ -4,22 +4,30 @@
 
 A step is one whole layer forward (router, top-k, dispatch, grouped SwiGLU GEMMs,
 weighted combine with the gated shared expert) over one batch of T tokens, inputs
-resident in HBM. Default workload: the Flash-Next-shaped decode layer (T=64, hidden 2560,
-512 experts top-10, inter 640, shared 640). Under torchrun each rank runs its own
-replica on its own token batch (weak scaling, no data-path collective); the time is the
-max over ranks of CUDA-event time.
+resident in HBM. By default the line's headline is the 2.4T-shaped prefill layer (T=8192,
+hidden 8192, 512 experts top-10, inter 2048, shared 2048) in tokens/s; the Flash-Next-shaped
+decode layer (T=64, reported in µs/layer), the Flash-Next-shaped prefill layer and the skewed
+2.4T-shaped layer (T=16384) are measured in the same run and reported under "workloads",
+each with its own clocks, roofline and error statistics. --workload NAME measures one
+workload only. Under torchrun each rank runs its own replica on its own token batch (weak
+scaling, no data-path collective); the time is the max over ranks of CUDA-event time.
 
-Reported beside the device-timed value:
+Reported for each workload beside the device-timed value:
 * e2e         -- the same metric through moe_layer_forward_host: pinned host x copied in,
                  layer, out copied back, every step inside the timed region;
-* roofline    -- the dominant kernel's algorithmic bytes per launch / its mean launch
-                 time (CUDA events on the launch stream), against the measured HBM copy
-                 bandwidth in MEASURED_PEAKS.json;
-* cpu_baseline-- the fp64 oracle on the host cores on a bounded token sample (rank 0, N=1);
-* clocks      -- nvidia-smi SM clocks and throttle reasons sampled during the timed region.
+* roofline    -- the dominant kernel's algorithmic bytes (or FLOPs) per launch / its mean
+                 launch time (CUDA events on the launch stream), against the measured peak
+                 in MEASURED_PEAKS.json;
+* layer       -- the whole layer's TC % (FLOPs / (peak x time)), HBM % (bytes / (bandwidth
+                 x time)) and roofline %, dense-equivalent and executed FLOPs separately;
+* errors      -- max |gpu - oracle| / RMS and mean relative error of the timed output on
+                 sampled tokens against the fp64 oracle, and the near-tie count;
+* cpu_baseline-- the fp64 oracle on the host cores on a bounded token sample (headline,
+                 rank 0, N=1);
+* clocks      -- nvidia-smi SM clocks and throttle reasons sampled during the timed regions.
 
 --impl reference times the oracle (the only other implementation of this layer) on the
-same workload on the host cores; under torchrun only rank 0 runs it.
+headline workload on the host cores; under torchrun only rank 0 runs it.
 """
 from __future__ import annotations
 
@@ -52,7 +60,7 @@ KERNEL_SOURCES = {  # kernel id -> source file whose hash a stored ncu traffic f
 }
 # oracle token sample per workload for the CPU baseline (about 10-30 s on a host)
 CPU_SAMPLE = {"tiny": 64, "flash_decode": 16, "flash_prefill": 32, "flash_prefill_e64": 32,
-              "t24_prefill_e16": 3, "t24_prefill": 3, "t24_skewed": 3}
+              "t24_prefill_e16": 2, "t24_prefill": 2, "t24_skewed": 2}
 
 
 def log(*a):
@@ -211,13 +219,15 @@ def oracle_sample(cfg, seed: int, ntok: int, fp8: bool = False):
     return host, x, gu, dn, rows
 
 
-def time_oracle(cfg, host, x, gu, dn) -> float:
+def time_oracle(cfg, host, x, gu, dn, with_result: bool = False):
+    """Seconds the oracle takes for the layer on the token rows x (and its result)."""
     import oracle
 
     t0 = time.perf_counter()
-    oracle.moe_forward(x, host.w_router, host.router_bias, gu.__getitem__, dn.__getitem__,
-                       host.ws_gate_up, host.ws_down, host.w_shared_gate, cfg.k)
-    return time.perf_counter() - t0
+    ref = oracle.moe_forward(x, host.w_router, host.router_bias, gu.__getitem__, dn.__getitem__,
+                             host.ws_gate_up, host.ws_down, host.w_shared_gate, cfg.k)
+    dt = time.perf_counter() - t0
+    return (dt, ref) if with_result else dt
 
 
 def blas_threads() -> int:
@@ -228,16 +238,6 @@ def blas_threads() -> int:
         return max(n) if n else 1
     except Exception:  # noqa: BLE001
         return os.cpu_count() or 1
-
-
-def cpu_baseline(cfg, seed=0, fp8=False):
-    ntok = CPU_SAMPLE.get(cfg.name, 8)
-    host, x, gu, dn, rows = oracle_sample(cfg, seed, ntok, fp8)
-    dt = time_oracle(cfg, host, x, gu, dn)
-    return {"value": len(rows) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{len(rows)} of {cfg.T} tokens of the {cfg.name} layer (seed {seed}), full layer per "
-                      f"token in fp64; expert weights made{' (FP8, dequantised)' if fp8 else ''} "
-                      f"before timing", "seconds": dt}
 
 
 # --------------------------------------------------------------------------- arms
@@ -320,7 +320,84 @@ def config_block(cfg, variant, timed_as="CUDA graph replay of one layer forward 
             "parallelism": "replicas: one token batch per GPU, no collective"}
 
 
-def run_ours(args, cfg, world, rank, local):
+def layer_totals(cfg, n_active: int, I_exec=None) -> dict:
+    """Algorithmic work of one layer forward: FLOPs of the expert GEMMs and the router
+    (dense-equivalent: every routed row at width I; executed: at the width the GEMMs ran,
+    I_exec after zero-channel compaction) and the bytes it must move at least (activated
+    routed experts, shared expert, router matrix, x in, out as fp32)."""
+    T, H, E, I, Is, R = cfg.T, cfg.H, cfg.E, cfg.I, cfg.Is, cfg.R
+    Ix = I if I_exec is None else I_exec
+    router = 2.0 * T * H * E
+    dense = 6.0 * (R * H * I + T * H * Is) + router
+    executed = 6.0 * (R * H * Ix + T * H * Is) + router
+    nbytes = (n_active * 3 * H * Ix + 3 * H * Is) * 2 + E * H * 4 + T * H * 2 + T * H * 4
+    return {"flops_dense_equivalent": dense, "flops_executed": executed, "bytes": float(nbytes)}
+
+
+def layer_fractions(tot: dict, seconds: float, peaks: dict) -> dict:
+    """TC % = F / (P t), HBM % = B / (BW t), roofline % = max(F / P, B / BW) / t."""
+    P = peaks["bf16_tflops"] * 1e12
+    Ps = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
+    BW = peaks["hbm_gbs"] * 1e9
+    F, B = tot["flops_executed"], tot["bytes"]
+    return {"tc_pct": 100.0 * F / (P * seconds), "tc_pct_of_sustained": 100.0 * F / (Ps * seconds),
+            "tc_pct_dense_equivalent": 100.0 * tot["flops_dense_equivalent"] / (P * seconds),
+            "hbm_pct": 100.0 * B / (BW * seconds),
+            "roofline_pct": 100.0 * max(F / P, B / BW) / seconds,
+            "bound": "tensor" if F / P > B / BW else "hbm",
+            "roofline_us": 1e6 * max(F / P, B / BW), **tot}
+
+
+def error_stats(gpu_out, gpu_ids, ref: dict, k: int) -> dict:
+    """Layer output against the fp64 oracle on the sampled tokens: max |d| / RMS(ref) and
+    sum |d| / sum |ref|; tokens whose id sets differ (near-ties) are counted and left out."""
+    import numpy as np
+
+    keep, ties = [], 0
+    for i in range(len(gpu_ids)):
+        if set(int(v) for v in gpu_ids[i]) == set(int(v) for v in ref["ids"][i]):
+            keep.append(i)
+        else:
+            ties += 1
+    g = np.asarray(gpu_out, dtype=np.float64)[keep]
+    r = np.asarray(ref["out"], dtype=np.float64)[keep]
+    d = np.abs(g - r)
+    rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
+    return {"tokens": len(gpu_ids), "max_abs_over_rms": float(d.max() / rms) if d.size else None,
+            "mean_rel": float(d.sum() / np.abs(r).sum()) if d.size else None,
+            "sample_id_sets_differ": ties,
+            "sample_near_ties_fp64": int(sum(1 for g_ in ref["gap"] if g_ < 1e-5)),
+            "tolerance": {"max_abs_over_rms": 1e-2, "mean_rel": 2e-3}}
+
+
+def kernel_roofline(kernels: dict, cfg, n_active: int, peaks: dict, peak_kind: str, fp8: bool,
+                    traffic_workload: str) -> dict:
+    """Roofline of the dominant kernel (largest total device time): algorithmic bytes (or
+    FLOPs) per launch over its mean launch time, against the measured peak."""
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
+    dom_bytes = algorithmic_bytes(dom, cfg, n_active, fp8)
+    bound = "tensor" if kernel_flops(dom, cfg) / max(dom_bytes, 1) > 290 else "hbm"
+    per_launch_s = kernels[dom]["ms_per_launch"] / 1e3
+    if bound == "hbm":
+        achieved = dom_bytes / per_launch_s / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved = kernel_flops(dom, cfg) / per_launch_s / 1e12
+        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+    return {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak,
+            "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+            "algorithmic_bytes_per_launch": dom_bytes,
+            "algorithmic_flops_per_launch": kernel_flops(dom, cfg),
+            "activated_experts": n_active,
+            "timed_from": "mean of the kernel's launch durations (CUDA events on its stream) over "
+                          "host-launched steps right after the graph-timed region",
+            "traffic": stored_traffic(dom + ("_fp8" if fp8 else ""), traffic_workload)}
+
+
+def measure_workload(args, cfg, world, rank, local, sampler, want_cpu_baseline: bool) -> dict:
+    """Everything the line reports for one workload: device-resident value, per-kernel
+    times, roofline, layer fractions, end-to-end value, clocks, errors against the oracle."""
     import numpy as np
     import torch
 
@@ -329,19 +406,16 @@ def run_ours(args, cfg, world, rank, local):
 
     variant = {"auto": moe.MOE_VARIANT_AUTO, "stream": moe.MOE_VARIANT_STREAM,
                "tc": moe.MOE_VARIANT_TC, "tc2": moe.MOE_VARIANT_TC2}[args.variant]
-    moe.moe_set_variant(variant)
+    full_cfg = cfg
     dev = synth.device_inputs(cfg, seed=0, x_seed=rank, device=f"cuda:{local}")
     compact = None
     if args.compact:
         # weight pre-pass (once, at load time): drop zero gate/up channels and their down
         # columns; the layer then runs with I = I_c
-        full_cfg = cfg
         t0 = time.time()
         dev, I_c = moe.compact_zero_channels(moe.shape_of(cfg), dev)
         torch.cuda.synchronize()
-        compact = {"I": cfg.I, "I_c": I_c, "prepass_s": round(time.time() - t0, 3),
-                   "dense_equivalent_flops": 6.0 * (full_cfg.R * full_cfg.H * full_cfg.I
-                                                    + full_cfg.T * full_cfg.H * full_cfg.Is)}
+        compact = {"I": cfg.I, "I_c": I_c, "prepass_s": round(time.time() - t0, 3)}
         cfg = cfg.replace(I=I_c)
         torch.cuda.empty_cache()
     s = moe.shape_of(cfg)
@@ -358,9 +432,10 @@ def run_ours(args, cfg, world, rank, local):
         dev["w_down"] = None
         torch.cuda.empty_cache()
         qs = moe.make_fp8_experts(q)
-    ws = moe.alloc_workspace(s, host_staging=True)
+    ws = moe.alloc_workspace(s, host_staging=True, variant=variant)
     out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
     ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
+    gap = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
     w = moe.make_weights(dev)
 
@@ -370,24 +445,27 @@ def run_ours(args, cfg, world, rank, local):
         st_ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
         st_w = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device="cuda")
         st_sg = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
+        st_gap = torch.empty((cfg.T,), dtype=torch.float32, device="cuda")
         st_off = torch.empty((cfg.E + 1,), dtype=torch.int32, device="cuda")
         st_tok = torch.empty((R,), dtype=torch.int32, device="cuda")
         st_ar = torch.empty((R,), dtype=torch.int32, device="cuda")
         st_y = torch.empty((R, cfg.H), dtype=torch.float32, device="cuda")
         st_ys = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
 
-    def layer(x_dev, out_dev, topk_ids=None):
+    def layer(x_dev, out_dev, topk_ids=None, gap_out=None):
         if fp8 is not None:
-            moe.moe_layer_forward_fp8(s, x_dev, w, qs, out_dev, ws, topk_ids=topk_ids)
+            moe.moe_layer_forward_fp8(s, x_dev, w, qs, out_dev, ws, topk_ids=topk_ids, gap=gap_out)
         elif args.staged:
-            moe.moe_router_topk(s, x_dev, w, st_ids, st_w, st_sg, None, ws)
+            moe.moe_router_topk(s, x_dev, w, st_ids, st_w, st_sg, st_gap, ws)
             moe.moe_permute(s, st_ids, st_off, st_tok, st_ar, ws)
             moe.moe_grouped_swiglu(s, x_dev, st_tok, st_off, w, st_y, st_ys, ws)
             moe.moe_unpermute_combine(s, st_y, st_ys, st_ar, st_w, st_sg, out_dev)
             if topk_ids is not None:
                 topk_ids.copy_(st_ids)
+            if gap_out is not None:
+                gap_out.copy_(st_gap)
         else:
-            moe.moe_layer_forward(s, x_dev, w, out_dev, ws, topk_ids=topk_ids)
+            moe.moe_layer_forward(s, x_dev, w, out_dev, ws, topk_ids=topk_ids, gap=gap_out)
 
     x_in = torch.empty_like(dev["x"])
     out_in = torch.empty_like(out)
@@ -400,35 +478,26 @@ def run_ours(args, cfg, world, rank, local):
         else:
             moe.moe_layer_forward_host(s, x_host, w, out_host, ws)
 
-    layer(dev["x"], out, topk_ids=ids)
+    layer(dev["x"], out, topk_ids=ids, gap_out=gap)
     st, flags = moe.moe_device_status(ws)
     if st != moe.MOE_OK:
-        raise RuntimeError(f"device status {st} ({flags})")
-    n_active = int(np.unique(ids.cpu().numpy()).size)
+        raise RuntimeError(f"{cfg.name}: device status {st} ({flags})")
+    ids_np = ids.cpu().numpy()
+    n_active = int(np.unique(ids_np).size)
+    counts = np.bincount(ids_np.ravel(), minlength=cfg.E)
+    near_ties_gpu = int((gap.cpu().numpy() < 1e-5).sum())
     for _ in range(args.warmup):
         layer(dev["x"], out)
     torch.cuda.synchronize()
 
-    props = torch.cuda.get_device_properties(local)
-    uuid = str(getattr(props, "uuid", ""))
-    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}") if rank == 0 else None
-    if sampler:
-        time.sleep(1.5)  # nvidia-smi start-up
-
-    def barrier():
-        dist_barrier(world)
-
-    def max_over_ranks(v: float) -> float:
-        return dist_max(v, world, "cuda")
-
     # ---- device-resident timed region: one layer forward per step, replayed from a CUDA
     # graph (as a served layer would run; --no-graph launches every kernel from the host)
-    windows = []
     graph = None
     moe.moe_profile_enable(True)  # fill the library's event pool before any capture
     layer(dev["x"], out)
     torch.cuda.synchronize()
     moe.moe_profile_collect()
+    per_step = None
     if not args.no_graph:
         graph = torch.cuda.CUDAGraph()
         n_cap = moe.moe_launch_count()
@@ -439,10 +508,11 @@ def run_ours(args, cfg, world, rank, local):
         for _ in range(2):
             graph.replay()
         torch.cuda.synchronize()
-    barrier()
+    dist_barrier(world)
     torch.cuda.synchronize()
     n0 = moe.moe_launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    windows = []
     w0 = time.time()
     e0.record(stream)
     for _ in range(args.steps):
@@ -463,11 +533,12 @@ def run_ours(args, cfg, world, rank, local):
         torch.cuda.synchronize()
     moe.moe_profile_enable(False)
     prof = moe.moe_profile_collect()
-    barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    dist_barrier(world)
+    ms = dist_max(e0.elapsed_time(e1), world, "cuda")
     st, flags = moe.moe_device_status(ws)
     if st != moe.MOE_OK:
-        raise RuntimeError(f"device status after the timed region {st} ({flags})")
+        raise RuntimeError(f"{cfg.name}: device status after the timed region {st} ({flags})")
+    out_np = out.cpu().numpy()  # the last timed step's output (same inputs every step)
 
     # ---- end to end through the host-buffer entry point
     x_host = dev["x"].cpu().pin_memory()
@@ -475,7 +546,7 @@ def run_ours(args, cfg, world, rank, local):
     for _ in range(max(1, min(args.warmup, 3))):
         layer_host(x_host, out_host)
     torch.cuda.synchronize()
-    barrier()
+    dist_barrier(world)
     w0 = time.time()
     e0.record(stream)
     for _ in range(args.steps):
@@ -483,17 +554,18 @@ def run_ours(args, cfg, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     windows.append((w0, time.time()))
-    barrier()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1))
-    if sampler:
-        sampler.stop()
+    dist_barrier(world)
+    ms_e2e = dist_max(e0.elapsed_time(e1), world, "cuda")
     st, flags = moe.moe_device_status(ws)
     if st != moe.MOE_OK:
-        raise RuntimeError(f"device status after timing {st} ({flags})")
+        raise RuntimeError(f"{cfg.name}: device status after timing {st} ({flags})")
+    del graph, ws, dev, w, out, out_in, x_in
+    if args.staged:
+        del st_y, st_ys
+    torch.cuda.empty_cache()
     if rank != 0:
         return None
 
-    value = job_value(cfg.T, args.steps, world, ms)
     peaks, peak_kind = load_peaks()
     kernels = {k: {"ms_per_launch": v[0] / v[1], "launches": v[1], "share": None}
                for k, v in prof.items() if v[1] > 0}
@@ -501,42 +573,54 @@ def run_ours(args, cfg, world, rank, local):
     for k, v in prof.items():
         if v[1] > 0:
             kernels[k]["share"] = v[0] / tot
-    dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
     is8 = fp8 is not None
-    dom_bytes = algorithmic_bytes(dom, cfg, n_active, is8)
-    bound = "tensor" if kernel_flops(dom, cfg) / max(dom_bytes, 1) > 290 else "hbm"
-    per_launch_s = kernels[dom]["ms_per_launch"] / 1e3
-    if bound == "hbm":
-        achieved = dom_bytes / per_launch_s / 1e9
-        peak, unit = peaks["hbm_gbs"], "GB/s"
-    else:
-        achieved = kernel_flops(dom, cfg) / per_launch_s / 1e12
-        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
-    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
-                "algorithmic_bytes_per_launch": dom_bytes,
-                "activated_experts": n_active,
-                "traffic": stored_traffic(dom + ("_fp8" if is8 else ""), cfg.name)}
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms / args.steps, "us_per_layer": 1e3 * ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3 (gate|up MMAs), bf16 (down MMAs)" if fp8 is not None else "bf16",
-            "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random router)",
-            "config": config_block(cfg, "fp8" if args.fp8 else
-                                   (args.variant + "+staged" if args.staged else args.variant),
-                                   "host launches of one layer forward per step" if args.no_graph
-                                   else "CUDA graph replay of one layer forward per step"),
-            "zero_channel_compaction": compact,
-            "fp8_experts": fp8,
-            "roofline": roofline,
-            "graph": not args.no_graph,
-            "e2e": {"value": job_value(cfg.T, args.steps, world, ms_e2e), "unit": "tokens/s",
-                    "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 4},
-            "gpu_launches": launches, "kernels": kernels,
-            "clocks": sampler.summary(windows) if sampler else None}
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(full_cfg if compact else cfg, fp8=fp8 is not None)
-    return line
+    seconds = ms / args.steps / 1e3
+    totals = layer_totals(full_cfg, n_active, I_exec=cfg.I)
+    if is8:  # routed experts at one byte per weight plus a 4-byte scale per row
+        totals["bytes"] = (n_active * (3 * cfg.H * cfg.I + 4 * (2 * cfg.I + cfg.H)) + 3 * cfg.H * cfg.Is * 2
+                           + cfg.E * cfg.H * 4 + cfg.T * cfg.H * 6)
+    res = {"workload": cfg.name, "value": job_value(cfg.T, args.steps, world, ms), "unit": "tokens/s",
+           "ms_per_step": ms / args.steps, "us_per_layer": 1e3 * ms / args.steps,
+           "steps": args.steps,
+           "config": config_block(full_cfg, "fp8" if args.fp8 else
+                                  (args.variant + "+staged" if args.staged else args.variant),
+                                  "host launches of one layer forward per step" if args.no_graph
+                                  else "CUDA graph replay of one layer forward per step"),
+           "zero_channel_compaction": compact, "fp8_experts": fp8,
+           "roofline": kernel_roofline(kernels, cfg, n_active, peaks, peak_kind, is8, cfg.name),
+           "layer": {**layer_fractions(totals, seconds, peaks), "peaks": f"{peak_kind} (MEASURED_PEAKS.json)"
+                     if peak_kind == "measured" else "fallback"},
+           "graph": not args.no_graph,
+           "e2e": {"value": job_value(cfg.T, args.steps, world, ms_e2e), "unit": "tokens/s",
+                   "h2d_bytes_per_step": cfg.T * cfg.H * 2, "d2h_bytes_per_step": cfg.T * cfg.H * 4},
+           "gpu_launches": launches, "kernels": kernels,
+           "expert_load": {"active": n_active, "max_rows": int(counts.max()),
+                           "mean_rows_active": float(counts[counts > 0].mean()),
+                           "min_rows_active": int(counts[counts > 0].min())},
+           "near_ties": {"tokens_gap_below_1e-5": near_ties_gpu,
+                         "note": "10th/11th logit gap of the kernel's own routing, all tokens"},
+           "clocks": sampler.summary(windows) if sampler else None}
+    # errors against the fp64 oracle on sampled tokens of the timed inputs (rank 0's batch);
+    # the oracle's time on the same sample is the CPU baseline
+    if not args.no_oracle and rank == 0:
+        ntok = ERROR_SAMPLE.get(full_cfg.name, 8)
+        host, x, gu, dn, rows = oracle_sample(full_cfg, 0, ntok, is8)
+        dt, ref = time_oracle(full_cfg, host, x, gu, dn, with_result=True)
+        res["errors"] = error_stats(out_np[rows], ids_np[rows], ref, cfg.k)
+        if want_cpu_baseline:
+            res["cpu_baseline"] = {
+                "value": len(rows) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{len(rows)} of {full_cfg.T} tokens of the {full_cfg.name} layer (seed 0), full "
+                          f"layer per token in fp64; expert weights made{' (FP8, dequantised)' if is8 else ''}"
+                          " before timing", "seconds": dt}
+    return res
+
+
+HEADLINE = "t24_prefill"
+SUITE = ("t24_prefill", "flash_decode", "flash_prefill", "t24_skewed")
+# tokens the oracle evaluates per workload for the error statistics (and the CPU baseline)
+ERROR_SAMPLE = {"tiny": 64, "flash_decode": 16, "flash_prefill": 16, "flash_prefill_e64": 16,
+                "flash_decode_e64": 16, "t24_prefill_e16": 4, "t24_prefill": 4, "t24_skewed": 4}
 
 
 def main():
@@ -544,12 +628,16 @@ def main():
 
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="flash_decode", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None, choices=sorted(synth.CONFIGS),
+                    help="one workload only (default: the 2.4T-shaped prefill layer as the "
+                         "headline, with the decode, Flash-Next prefill and skewed layers beside it)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto", choices=["auto", "stream", "tc", "tc2"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-oracle", action="store_true",
+                    help="skip the oracle error statistics and the CPU baseline")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel from the host")
     ap.add_argument("--staged", action="store_true",
                     help="time the four stage entry points (y in fp32, separate combine) "
@@ -560,21 +648,65 @@ def main():
                     help="zero-channel compaction of the routed experts before timing (weight pre-pass)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    cfg = synth.CONFIGS[args.workload]
+    if args.staged and (args.fp8 or args.compact):
+        ap.error("--staged times the bf16 stage entry points on the full bank: "
+                 "it does not combine with --fp8 or --compact")
+    if args.no_oracle:
+        args.no_cpu_baseline = True
+    names = [args.workload] if args.workload else list(SUITE)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
-        line = run_reference(args, cfg, world, rank)
-    else:
-        world, rank, local = dist_setup()
-        line = run_ours(args, cfg, world, rank, local)
+        line = run_reference(args, synth.CONFIGS[names[0]], world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+
+    world, rank, local = dist_setup()
+    sampler = None
+    if rank == 0:
+        props = torch.cuda.get_device_properties(local)
+        uuid = str(getattr(props, "uuid", ""))
+        sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+        time.sleep(1.5)  # nvidia-smi start-up
+    results = []
+    try:
+        for i, name in enumerate(names):
+            results.append(measure_workload(args, synth.CONFIGS[name], world, rank, local, sampler,
+                                            want_cpu_baseline=(i == 0 and world == 1
+                                                               and not args.no_cpu_baseline)))
+    finally:
+        if sampler:
+            sampler.stop()
         if world > 1:
             import torch.distributed as dist
 
             dist.destroy_process_group()
-    if line is not None:
-        print(json.dumps(line), flush=True)
+    if rank != 0:
+        return
+    head = results[0]
+    line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "us_per_layer": head["us_per_layer"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "e4m3 (gate|up MMAs), bf16 (down MMAs)" if args.fp8 else "bf16",
+            "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random "
+                    "router; the skewed layer adds a Zipf(1.1) router bias and 71% zero gate/up channels)"}
+    for key in ("config", "roofline", "layer", "e2e", "gpu_launches", "kernels", "clocks", "errors",
+                "near_ties", "expert_load", "cpu_baseline", "zero_channel_compaction", "fp8_experts",
+                "graph"):
+        if key in head:
+            line[key] = head[key]
+    if len(results) > 1:
+        line["gpu_launches"] = sum(r["gpu_launches"] for r in results)
+        line["gpu_launches_note"] = "all workloads' timed regions (the headline's alone: " \
+                                    f"{head['gpu_launches']})"
+        line["workloads"] = {r["workload"]: {k: v for k, v in r.items() if k not in ("workload",)}
+                             for r in results[1:]}
+    print(json.dumps(line), flush=True)
 
 
 if __name__ == "__main__":

@@ -82,3 +82,48 @@ def test_reference_arm_times_the_fp8_oracle():
     line = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][-1])
     assert line["impl"] == "reference" and line["config"]["variant"] == "fp8"
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_layer_totals_match_the_survey_counts():
+    # 2.4T-shaped prefill, every expert active: routed 8.246 TFLOP + shared 0.825 TFLOP +
+    # router 68.7 GFLOP; 51.54 GB of routed weights + shared expert + router matrix + x + out
+    # (fp32) = 52.06 GB
+    cfg = synth.CONFIGS["t24_prefill"]
+    t = bench.layer_totals(cfg, 512)
+    assert t["flops_dense_equivalent"] == t["flops_executed"]
+    assert t["flops_dense_equivalent"] == pytest.approx(8.246e12 + 0.825e12 + 68.7e9, rel=1e-3)
+    assert t["bytes"] == pytest.approx(52.06e9, rel=1e-3)
+    # zero-channel compaction to I_c = 640: executed routed FLOPs scale by 640 / 2048,
+    # dense-equivalent FLOPs do not change
+    c = bench.layer_totals(synth.CONFIGS["t24_skewed"], 512, I_exec=640)
+    full = bench.layer_totals(synth.CONFIGS["t24_skewed"], 512)
+    cfg5 = synth.CONFIGS["t24_skewed"]
+    routed = 6.0 * cfg5.R * cfg5.H * cfg5.I
+    assert c["flops_dense_equivalent"] == full["flops_dense_equivalent"]
+    assert full["flops_executed"] - c["flops_executed"] == pytest.approx(routed * (1 - 640 / 2048))
+
+
+def test_layer_fractions_by_hand():
+    tot = {"flops_dense_equivalent": 2e12, "flops_executed": 1e12, "bytes": 4e9}
+    peaks = {"bf16_tflops": 1000.0, "bf16_tflops_sustained": 800.0, "hbm_gbs": 2000.0}
+    f = bench.layer_fractions(tot, 0.004, peaks)  # 4 ms
+    assert f["tc_pct"] == pytest.approx(25.0)      # 1 TFLOP / (1 PFLOP/s x 4 ms)
+    assert f["tc_pct_of_sustained"] == pytest.approx(31.25)
+    assert f["tc_pct_dense_equivalent"] == pytest.approx(50.0)
+    assert f["hbm_pct"] == pytest.approx(50.0)     # 4 GB / (2 TB/s x 4 ms)
+    assert f["roofline_pct"] == pytest.approx(50.0) and f["bound"] == "hbm"
+    assert f["roofline_us"] == pytest.approx(2000.0)
+
+
+def test_error_stats_leave_out_differing_id_sets():
+    import numpy as np
+
+    ref = {"out": np.array([[1.0, -1.0], [2.0, 2.0], [5.0, 5.0]]),
+           "ids": np.array([[0, 1], [2, 3], [4, 5]]), "gap": np.array([1.0, 1.0, 1e-6])}
+    gpu = np.array([[1.01, -1.0], [2.0, 2.0], [0.0, 0.0]])
+    ids = np.array([[1, 0], [3, 2], [4, 6]])  # last token: a near-tie chose another set
+    e = bench.error_stats(gpu, ids, ref, 2)
+    rms = np.sqrt((1 + 1 + 4 + 4) / 4)
+    assert e["sample_id_sets_differ"] == 1 and e["sample_near_ties_fp64"] == 1
+    assert e["max_abs_over_rms"] == pytest.approx(0.01 / rms)
+    assert e["mean_rel"] == pytest.approx(0.01 / 6.0)
