@@ -98,7 +98,9 @@ typedef enum moe_kernel {
 
 /* Bytes of device workspace the calls below need for `shape` (0 on a bad shape).
  * One workspace serves all calls; its first bytes hold the device status word.
- * Calls that share a workspace must not overlap in time on the GPU. */
+ * The size never decreases as T grows, so a workspace sized for T serves every smaller
+ * batch with the same H, E, k, I, Is. Calls that share a workspace must not overlap in
+ * time on the GPU. */
 size_t moe_workspace_bytes(const moe_shape* shape);
 
 /* Extra bytes moe_layer_forward_host needs on top of moe_workspace_bytes
@@ -169,6 +171,9 @@ moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_ids, 
  * sorted_token / offsets as produced by moe_permute. The intermediate
  * h = SiLU(gate) * up is carried as a pair of bf16 values (hi = bf16(h), lo = bf16(h - hi),
  * about 16 significant bits) into the down projection; accumulation is fp32.
+ * With weights->ws_gate_up and weights->ws_down both NULL there is no shared expert in this
+ * call (the routed experts of an expert-parallel owner, below): y_shared is not written and
+ * may be NULL.
  */
 moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const int32_t* sorted_token,
                               const int32_t* offsets, const moe_weights* weights, float* y,
@@ -204,6 +209,54 @@ moe_status moe_layer_forward(const moe_shape* shape, const void* x, const moe_we
 moe_status moe_layer_forward_host(const moe_shape* shape, const void* x_host,
                                   const moe_weights* weights, float* out_host, void* ws,
                                   size_t ws_bytes, void* stream);
+
+/*
+ * Expert parallelism ("Qwen3.8-Flash-Next" architecture study, section "Expert
+ * parallelism": the routed experts are split across GPUs, and dispatch and combine
+ * exchange token activations across expert owners). The E routed experts are split into G
+ * contiguous slices of E_local = E / G, slice d owned by rank d. moe_permute's packed order
+ * (experts ascending) is then already grouped by owner. The exchange itself, an all-to-all
+ * of variable-size blocks of rows, belongs to the caller's collective library (NCCL through
+ * torch.distributed in the Python binding); these calls move rows and plans on one GPU
+ * around it. One layer step on rank r:
+ *   holder:  moe_router_topk, moe_permute (all E experts), moe_ep_counts,
+ *            moe_gather_rows(index = sorted_token)            -> send buffer
+ *   exchange counts [G][E_local], then rows (sizes from the counts)
+ *   owner:   moe_ep_regroup, moe_grouped_swiglu(T = received rows, k = 1, E = E_local,
+ *            x = received rows, sorted_token = src_index, no shared expert),
+ *            moe_scatter_rows(index = src_index)            -> rows back in received order
+ *   exchange the output rows back (reverse sizes)
+ *   holder:  shared expert (moe_grouped_swiglu with every routed group empty) and
+ *            moe_unpermute_combine on the returned rows, which are in its packed order.
+ *
+ * moe_ep_counts: offsets int32 [G*E_local + 1] from moe_permute -> counts int32
+ *   [G][E_local] (rows for owner d's local expert e) and rows int32 [G] (all rows for owner d).
+ * moe_gather_rows: out[p] = x[index[p]] for p < rows; x, out bf16 rows of H elements (H a
+ *   multiple of 8); index int32 in [0, n_src).
+ * moe_ep_regroup: on an owner, recv_counts int32 [G][E_local] (rows source s sent for local
+ *   expert e; the received buffer holds, source by source, each source's rows expert by
+ *   expert). Writes offsets int32 [E_local + 1] of the expert-major order, src_index int32
+ *   [capacity] (expert-major row p is received row src_index[p]) and, if not NULL,
+ *   src_rows int32 [G] (rows received from each source). G * E_local <= 1024; more rows
+ *   than capacity are dropped and flagged.
+ * moe_scatter_rows: out[index[p]] = y[p] for p < rows; y, out fp32 rows of H elements (H a
+ *   multiple of 4); index int32 in [0, n_dst).
+ * ws (optional, may be NULL): a workspace whose status word records an index or count out
+ * of range (moe_device_status then reports MOE_ERR_DEVICE_BOUNDS); such rows are skipped.
+ * Errors: MOE_ERR_INVALID_ARG (bad size, null or misaligned pointer), MOE_ERR_UNSUPPORTED,
+ * MOE_ERR_CUDA. All asynchronous on `stream`.
+ */
+moe_status moe_ep_counts(int32_t G, int32_t E_local, const int32_t* offsets, int32_t* counts,
+                         int32_t* rows, void* stream);
+moe_status moe_gather_rows(int64_t rows, int32_t H, const void* x, int64_t n_src,
+                           const int32_t* index, void* out, void* ws, size_t ws_bytes,
+                           void* stream);
+moe_status moe_ep_regroup(int32_t G, int32_t E_local, const int32_t* recv_counts,
+                          int64_t capacity, int32_t* offsets, int32_t* src_index,
+                          int32_t* src_rows, void* ws, size_t ws_bytes, void* stream);
+moe_status moe_scatter_rows(int64_t rows, int32_t H, const float* y, int64_t n_dst,
+                            const int32_t* index, float* out, void* ws, size_t ws_bytes,
+                            void* stream);
 
 /*
  * Zero-channel compaction of structurally sparse routed experts: a weight pre-pass run once

@@ -82,6 +82,12 @@ _SIGS = {
     "moe_quantize_fp8_experts": ([_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "moe_layer_forward_fp8": ([_SP, _vp, _WP, _FP, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
                               ctypes.c_int),
+    "moe_ep_counts": ([_i32, _i32, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moe_gather_rows": ([ctypes.c_int64, _i32, _vp, ctypes.c_int64, _vp, _vp, _vp, _sz, _vp],
+                        ctypes.c_int),
+    "moe_ep_regroup": ([_i32, _i32, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
+    "moe_scatter_rows": ([ctypes.c_int64, _i32, _vp, ctypes.c_int64, _vp, _vp, _vp, _sz, _vp],
+                         ctypes.c_int),
     "moe_set_variant": ([ctypes.c_int], ctypes.c_int),
     "moe_workspace_set_variant": ([_vp, _sz, ctypes.c_int], ctypes.c_int),
     "moe_compact_workspace_bytes": ([_SP], _sz),
@@ -270,6 +276,32 @@ def moe_layer_forward_fp8(shape, x, weights, experts, out, ws, topk_ids=None, to
                                       ctypes.byref(q), _ptr(out), _ptr(topk_ids), _ptr(topk_w),
                                       _ptr(gap), _ptr(ws), _nbytes(ws), _stream(stream)),
            "moe_layer_forward_fp8")
+
+
+def _ws_args(ws):
+    return (None, 0) if ws is None else (_ptr(ws), _nbytes(ws))
+
+
+def moe_ep_counts(G: int, E_local: int, offsets, counts, rows, stream=None) -> None:
+    _check(_lib.moe_ep_counts(int(G), int(E_local), _ptr(offsets), _ptr(counts), _ptr(rows),
+                              _stream(stream)), "moe_ep_counts")
+
+
+def moe_gather_rows(rows: int, H: int, x, n_src: int, index, out, ws=None, stream=None) -> None:
+    _check(_lib.moe_gather_rows(int(rows), int(H), _ptr(x), int(n_src), _ptr(index), _ptr(out),
+                                *_ws_args(ws), _stream(stream)), "moe_gather_rows")
+
+
+def moe_ep_regroup(G: int, E_local: int, recv_counts, capacity: int, offsets, src_index,
+                   src_rows=None, ws=None, stream=None) -> None:
+    _check(_lib.moe_ep_regroup(int(G), int(E_local), _ptr(recv_counts), int(capacity),
+                               _ptr(offsets), _ptr(src_index), _ptr(src_rows), *_ws_args(ws),
+                               _stream(stream)), "moe_ep_regroup")
+
+
+def moe_scatter_rows(rows: int, H: int, y, n_dst: int, index, out, ws=None, stream=None) -> None:
+    _check(_lib.moe_scatter_rows(int(rows), int(H), _ptr(y), int(n_dst), _ptr(index), _ptr(out),
+                                 *_ws_args(ws), _stream(stream)), "moe_scatter_rows")
 
 
 def moe_set_variant(variant: int) -> None:

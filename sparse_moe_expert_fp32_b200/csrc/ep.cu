@@ -6,6 +6,7 @@
 // With the experts split into G contiguous slices of E/G, the dispatch order of
 // moe_permute (packed rows grouped by expert, experts ascending) is already grouped by
 // owner rank: rank d's rows are packed rows [offsets[d E/G], offsets[(d+1) E/G]). So:
+//   ep_counts_kernel      per owner rank and local expert, the row counts to send;
 //   gather_rows_kernel    the send buffer: token rows in packed order, xs[p] = x[index[p]];
 //   ep_regroup_kernel     on the owner, after the exchange: the received rows arrive
 //                         grouped by source rank, then by expert; this builds the
@@ -63,6 +64,17 @@ scatter_rows_f32_kernel(const float* __restrict__ y, const int32_t* __restrict__
   }
 }
 
+// On the rank holding the tokens: counts[d][e] = rows of owner d's local expert e
+// (packed rows of expert d El + e), rows[d] = all of owner d's rows, from moe_permute's
+// offsets. One CTA of kScanThreads.
+__global__ void __launch_bounds__(kScanThreads)
+ep_counts_kernel(const int32_t* __restrict__ offsets, int G, int El, int32_t* __restrict__ counts,
+                 int32_t* __restrict__ rows) {
+  const int i = threadIdx.x;
+  if (i < G * El) counts[i] = offsets[i + 1] - offsets[i];
+  if (i < G) rows[i] = offsets[(i + 1) * El] - offsets[i * El];
+}
+
 // counts[s][e] = rows source rank s sent for local expert e (G x El <= kMaxE, one CTA of
 // kScanThreads). The received buffer holds, source by source, each source's rows for
 // expert 0, then expert 1, ...: segment (s, e) starts at seg(s, e), the exclusive prefix
@@ -72,7 +84,7 @@ scatter_rows_f32_kernel(const float* __restrict__ y, const int32_t* __restrict__
 __global__ void __launch_bounds__(kScanThreads)
 ep_regroup_kernel(const int32_t* __restrict__ counts, int G, int El, int64_t capacity,
                   int32_t* __restrict__ offsets, int32_t* __restrict__ src_index,
-                  uint32_t* __restrict__ status) {
+                  int32_t* __restrict__ src_rows, uint32_t* __restrict__ status) {
   __shared__ int smem[33];
   __shared__ int cnt[kMaxE];
   __shared__ int seg[kMaxE];
@@ -97,6 +109,10 @@ ep_regroup_kernel(const int32_t* __restrict__ counts, int G, int El, int64_t cap
   if (i < n) dst[i] = b;
   __syncthreads();
   if (i < El) offsets[i] = dst[i * G];
+  if (src_rows && i < G) {  // rows received from source i
+    const int end = (i + 1 < G) ? seg[(i + 1) * El] : total;
+    src_rows[i] = end - seg[i * El];
+  }
   if (i == 0) {
     offsets[El] = (int64_t)total < capacity ? total : (int)capacity;
     if ((int64_t)total > capacity) set_flag(status, kFlagBounds);
@@ -135,11 +151,18 @@ cudaError_t launch_scatter_rows_f32(const float* y, const int32_t* index, int64_
 }
 
 cudaError_t launch_ep_regroup(const int32_t* counts, int G, int El, int64_t capacity,
-                              int32_t* offsets, int32_t* src_index, uint32_t* status,
-                              cudaStream_t st) {
+                              int32_t* offsets, int32_t* src_index, int32_t* src_rows,
+                              uint32_t* status, cudaStream_t st) {
   LaunchScope scope(MOE_K_PERMUTE, st);
   ep_regroup_kernel<<<1, kScanThreads, 0, st>>>(counts, G, El, capacity, offsets, src_index,
-                                                status);
+                                                src_rows, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_counts(const int32_t* offsets, int G, int El, int32_t* counts,
+                             int32_t* rows, cudaStream_t st) {
+  LaunchScope scope(MOE_K_PERMUTE, st);
+  ep_counts_kernel<<<1, kScanThreads, 0, st>>>(offsets, G, El, counts, rows);
   return cudaGetLastError();
 }
 

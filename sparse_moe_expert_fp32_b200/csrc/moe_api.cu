@@ -26,7 +26,10 @@ Layout layout(const moe_shape& s) {
     return at;
   };
   L.status = take(64 * sizeof(uint32_t));
-  L.logits = take((T < 512 ? 4 : 1) * T * E * sizeof(float));
+  // below 512 tokens the router keeps four partial sums per logit; the region is sized so
+  // that the workspace never shrinks as T grows (a workspace for T serves every T' <= T)
+  const size_t logit_rows = T < 512 ? 4 * T : (T > 2044 ? T : 2044);
+  L.logits = take(logit_rows * E * sizeof(float));
   L.wr_split = take(E * 3 * H * sizeof(uint16_t));
   L.ids = take(R * sizeof(int32_t));
   L.w = take(R * sizeof(float));
@@ -508,15 +511,25 @@ moe_status moe_scatter_rows(int64_t rows, int32_t H, const float* y, int64_t n_d
   return MOE_OK;
 }
 
+moe_status moe_ep_counts(int32_t G, int32_t E_local, const int32_t* offsets, int32_t* counts,
+                         int32_t* rows, void* stream) {
+  if (G <= 0 || E_local <= 0) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)G * E_local > kMaxE) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(offsets) || !aligned16(counts) || !aligned16(rows)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(launch_ep_counts(offsets, G, E_local, counts, rows, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
 moe_status moe_ep_regroup(int32_t G, int32_t E_local, const int32_t* recv_counts,
-                          int64_t capacity, int32_t* offsets, int32_t* src_index, void* ws,
-                          size_t ws_bytes, void* stream) {
+                          int64_t capacity, int32_t* offsets, int32_t* src_index,
+                          int32_t* src_rows, void* ws, size_t ws_bytes, void* stream) {
   if (G <= 0 || E_local <= 0 || capacity < 0) return MOE_ERR_INVALID_ARG;
   if ((int64_t)G * E_local > kMaxE || capacity >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
-  if (!aligned16(recv_counts) || !aligned16(offsets) || (capacity > 0 && !aligned16(src_index)))
+  if (!aligned16(recv_counts) || !aligned16(offsets) || (capacity > 0 && !aligned16(src_index)) ||
+      (src_rows && !aligned16(src_rows)))
     return MOE_ERR_INVALID_ARG;
   if (ws && (!aligned16(ws) || ws_bytes < 256)) return MOE_ERR_INVALID_ARG;
-  MOE_CUDA(launch_ep_regroup(recv_counts, G, E_local, capacity, offsets, src_index,
+  MOE_CUDA(launch_ep_regroup(recv_counts, G, E_local, capacity, offsets, src_index, src_rows,
                              static_cast<uint32_t*>(ws), (cudaStream_t)stream));
   return MOE_OK;
 }

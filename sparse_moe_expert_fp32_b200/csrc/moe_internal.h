@@ -23,6 +23,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Layout {
   size_t status;        // uint32 [64]: [0] = error flags, [1..] = diagnostics
   size_t logits;        // fp32 [4][T][E] partial router logits for T < 512, else [T][E]
+                        // (at least 2044 x E entries from T = 512 on: sizes grow with T)
   size_t wr_split;      // bf16 [E][3H]: router matrix as hi|mid|lo bf16 pieces (tensor-core router)
   size_t ids;           // int32 [T][k]
   size_t w;             // fp32 [T][k]
@@ -122,8 +123,10 @@ cudaError_t launch_scatter_rows_f32(const float* y, const int32_t* index, int64_
                                     int64_t n_dst, int H, float* out, uint32_t* status, int sms,
                                     cudaStream_t st);
 cudaError_t launch_ep_regroup(const int32_t* counts, int G, int El, int64_t capacity,
-                              int32_t* offsets, int32_t* src_index, uint32_t* status,
-                              cudaStream_t st);
+                              int32_t* offsets, int32_t* src_index, int32_t* src_rows,
+                              uint32_t* status, cudaStream_t st);
+cudaError_t launch_ep_counts(const int32_t* offsets, int G, int El, int32_t* counts,
+                             int32_t* rows, cudaStream_t st);
 cudaError_t launch_stream_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                                   const int32_t* sorted_token, const moe_weights& w,
                                   cudaStream_t st);

@@ -155,3 +155,13 @@ def test_fp8_entry_points_reject_bad_pointers_before_launch():
     assert L.moe_quantize_fp8_experts(ctypes.byref(s), 16, 32, 48, 64, 80, 100,
                                       None) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_launch_count() == before
+
+
+@pytest.mark.parametrize("E,k", [(512, 10), (64, 1), (16, 4)])
+def test_workspace_size_never_shrinks_as_the_batch_grows(E, k):
+    # a workspace sized for the largest batch must serve every smaller one
+    prev = 0
+    for T in list(range(1, 3000, 7)) + [4095, 4096, 8192]:
+        n = moe.moe_workspace_bytes(moe.make_shape(T, 256, E, k, 128, 128))
+        assert n >= prev, T
+        prev = n
