@@ -136,18 +136,20 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- roofline
 
-def algorithmic_bytes(kernel: str, cfg, n_active: int, fp8: bool = False) -> float:
+def algorithmic_bytes(kernel: str, cfg, n_active: int, fp8: bool = False, h_bytes: int = 4) -> float:
     """Bytes a launch of `kernel` must move at least (each operand once). fp8: the routed
-    experts as E4M3 codes (1 byte per weight) plus one fp32 scale per weight row."""
+    experts as E4M3 codes (1 byte per weight) plus one fp32 scale per weight row. h_bytes:
+    bytes per element of the intermediate h (4: the bf16 pair hi + lo; 2: one fp16 value,
+    with the fp16 down operands)."""
     T, H, I, Is, R = cfg.T, cfg.H, cfg.I, cfg.Is, cfg.R
     if fp8 and kernel == "gate_up":
         return n_active * 2 * I * (H + 4) + (2 * Is * H + T * H) * 2 + (R * I + T * Is) * 4
     if fp8 and kernel == "down":
         return n_active * H * (I + 4) + H * Is * 2 + (R * I + T * Is) * 4 + T * H * 4
-    if kernel == "gate_up":  # activated experts' gate|up + shared gate|up + x + h (hi+lo bf16)
-        return (n_active * 2 * I * H + 2 * Is * H + T * H) * 2 + (R * I + T * Is) * 4
-    if kernel == "down":  # activated experts' down + shared down + h (hi+lo) in + out (fp32)
-        return (n_active * H * I + H * Is) * 2 + (R * I + T * Is) * 4 + T * H * 4
+    if kernel == "gate_up":  # activated experts' gate|up + shared gate|up + x + h out
+        return (n_active * 2 * I * H + 2 * Is * H + T * H) * 2 + (R * I + T * Is) * h_bytes
+    if kernel == "down":  # activated experts' down + shared down + h in + out (fp32)
+        return (n_active * H * I + H * Is) * 2 + (R * I + T * Is) * h_bytes + T * H * 4
     if kernel == "router_logits":
         return cfg.E * H * 4 + T * H * 2 + T * cfg.E * 4
     if kernel == "router_topk":
@@ -371,11 +373,11 @@ def error_stats(gpu_out, gpu_ids, ref: dict, k: int) -> dict:
 
 
 def kernel_roofline(kernels: dict, cfg, n_active: int, peaks: dict, peak_kind: str, fp8: bool,
-                    traffic_workload: str) -> dict:
+                    traffic_workload: str, h_bytes: int = 4) -> dict:
     """Roofline of the dominant kernel (largest total device time): algorithmic bytes (or
     FLOPs) per launch over its mean launch time, against the measured peak."""
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_launch"] * kernels[k]["launches"])
-    dom_bytes = algorithmic_bytes(dom, cfg, n_active, fp8)
+    dom_bytes = algorithmic_bytes(dom, cfg, n_active, fp8, h_bytes)
     bound = "tensor" if kernel_flops(dom, cfg) / max(dom_bytes, 1) > 290 else "hbm"
     per_launch_s = kernels[dom]["ms_per_launch"] / 1e3
     if bound == "hbm":
@@ -392,7 +394,8 @@ def kernel_roofline(kernels: dict, cfg, n_active: int, peaks: dict, peak_kind: s
             "activated_experts": n_active,
             "timed_from": "mean of the kernel's launch durations (CUDA events on its stream) over "
                           "host-launched steps right after the graph-timed region",
-            "traffic": stored_traffic(dom + ("_fp8" if fp8 else ""), traffic_workload)}
+            "traffic": stored_traffic(dom + ("_fp8" if fp8 else ("_f16" if h_bytes == 2 else "")),
+                                      traffic_workload)}
 
 
 def measure_workload(args, cfg, world, rank, local, sampler, want_cpu_baseline: bool) -> dict:
@@ -432,6 +435,17 @@ def measure_workload(args, cfg, world, rank, local, sampler, want_cpu_baseline: 
         dev["w_down"] = None
         torch.cuda.empty_cache()
         qs = moe.make_fp8_experts(q)
+    down_f16 = None
+    if fp8 is None and not args.down_bf16_pair and args.variant != "stream":
+        # weight pre-pass (once, at load time): the down matrices re-encoded as fp16(W * 2^8)
+        # so that the down GEMM takes h as one fp16 value (one MMA per K step)
+        t0 = time.time()
+        dev = moe.prepare_down_f16(s, dev)
+        torch.cuda.synchronize()
+        down_f16 = {"prepass_s": round(time.time() - t0, 3),
+                    "weights": "W_down re-encoded once as fp16(W * 2^8): exact for 2^-25 <= |w| < 256",
+                    "h": "fp16(h * 2^-8): 11 significant bits for |h| >= 2^-6 (the bf16 pair hi + lo "
+                         "carries 16); fp32 accumulation"}
     ws = moe.alloc_workspace(s, host_staging=True, variant=variant)
     out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
     ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
@@ -586,8 +600,9 @@ def measure_workload(args, cfg, world, rank, local, sampler, want_cpu_baseline: 
                                   (args.variant + "+staged" if args.staged else args.variant),
                                   "host launches of one layer forward per step" if args.no_graph
                                   else "CUDA graph replay of one layer forward per step"),
-           "zero_channel_compaction": compact, "fp8_experts": fp8,
-           "roofline": kernel_roofline(kernels, cfg, n_active, peaks, peak_kind, is8, cfg.name),
+           "zero_channel_compaction": compact, "fp8_experts": fp8, "down_operands_fp16": down_f16,
+           "roofline": kernel_roofline(kernels, cfg, n_active, peaks, peak_kind, is8, cfg.name,
+                                       h_bytes=2 if down_f16 else 4),
            "layer": {**layer_fractions(totals, seconds, peaks), "peaks": f"{peak_kind} (MEASURED_PEAKS.json)"
                      if peak_kind == "measured" else "fallback"},
            "graph": not args.no_graph,
@@ -646,6 +661,9 @@ def main():
                     help="routed experts in FP8 (E4M3 + fp32 row scales, quantised before timing)")
     ap.add_argument("--compact", action="store_true",
                     help="zero-channel compaction of the routed experts before timing (weight pre-pass)")
+    ap.add_argument("--down-bf16-pair", action="store_true",
+                    help="keep the down GEMM on the bf16 weights with h as the bf16 pair hi + lo "
+                         "(default: the fp16 down-operand pre-pass runs before timing)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.staged and (args.fp8 or args.compact):
@@ -692,12 +710,15 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
             "us_per_layer": head["us_per_layer"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "e4m3 (gate|up MMAs), bf16 (down MMAs)" if args.fp8 else "bf16",
+            "dtype": ("e4m3 (gate|up MMAs), bf16 (down MMAs)" if args.fp8 else
+                      "bf16 (router split, gate|up MMAs)" + ("" if head.get("down_operands_fp16") is None
+                                                             else ", fp16 (down MMAs)")
+                      + ", fp32 accumulation and output"),
             "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random "
                     "router; the skewed layer adds a Zipf(1.1) router bias and 71% zero gate/up channels)"}
     for key in ("config", "roofline", "layer", "e2e", "gpu_launches", "kernels", "clocks", "errors",
                 "near_ties", "expert_load", "cpu_baseline", "zero_channel_compaction", "fp8_experts",
-                "graph"):
+                "down_operands_fp16", "graph"):
         if key in head:
             line[key] = head[key]
     if len(results) > 1:

@@ -50,7 +50,8 @@ typedef enum moe_status {
   MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < moe_workspace_bytes(shape)         */
   MOE_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed          */
   MOE_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device-side wait gave up            */
-  MOE_ERR_DEVICE_BOUNDS = 6        /* a kernel met an expert id outside [0, E)      */
+  MOE_ERR_DEVICE_BOUNDS = 6,       /* a kernel met an expert id outside [0, E)      */
+  MOE_ERR_DEVICE_RANGE = 7         /* a value saturated to fit fp16 (down operands)  */
 } moe_status;
 
 /* Layer shape. T tokens, hidden size H, E routed experts, k experts per token,
@@ -68,6 +69,9 @@ typedef struct moe_weights {
   const void* ws_gate_up;   /* bf16 [2Is][H]   shared expert gate|up                      */
   const void* ws_down;      /* bf16 [H][Is]    shared expert down                          */
   const void* w_shared_gate;/* bf16 [H]        shared-expert output gate vector            */
+  /* Optional fp16 down operands from moe_prepare_down_f16, or NULL (both or neither): */
+  const void* w_down_f16;   /* fp16 [E][H][I]  fp16(w_down * 2^8)                          */
+  const void* ws_down_f16;  /* fp16 [H][Is]    fp16(ws_down * 2^8)                         */
 } moe_weights;
 
 /* Grouped-GEMM variant used by moe_grouped_swiglu and moe_layer_forward. */
@@ -293,6 +297,28 @@ moe_status moe_zero_channel_count(const moe_shape* shape, const void* w_gate_up,
 moe_status moe_compact_zero_channels(const moe_shape* shape, const void* w_gate_up,
                                      const void* w_down, int32_t I_c, void* gate_up_c,
                                      void* down_c, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * fp16 down operands: a weight pre-pass, run once when the weights are loaded. The down
+ * projection y = W_down h can take h as one fp16 value per element (11 significant bits)
+ * instead of the bf16 pair hi + lo (16 bits): one MMA per K step instead of two, and down
+ * tiles of up to 256 token rows. The tensor core's f16 MMA needs both operands in one
+ * format, so the down matrices are re-encoded as W' = fp16(W * 2^8); the layer then stores
+ * h' = fp16(h * 2^-8), and W' h' = W h. A bf16 weight w with 2^-25 <= |w| < 256 (or 0) is
+ * re-encoded exactly; smaller magnitudes round with an error of at most 2^-33; larger ones
+ * saturate and set the range flag. An intermediate |h| above 65504 * 2^8 saturates and sets
+ * the range flag too (moe_device_status: MOE_ERR_DEVICE_RANGE).
+ * moe_prepare_down_f16: w_down bf16 [E][H][I] -> w_down_f16 fp16 [E][H][I]; ws_down bf16
+ *   [H][Is] -> ws_down_f16 fp16 [H][Is]; asynchronous on `stream`. ws (optional, may be
+ *   NULL) receives the range flag in its status word.
+ * Pass the results as moe_weights.w_down_f16 / ws_down_f16: moe_layer_forward,
+ * moe_layer_forward_host and moe_grouped_swiglu then use them whenever they take the
+ * tensor-core kernels (the down GEMM then runs on CTA pairs); the weight-streaming variant
+ * ignores them. Outputs stay fp32 with fp32 accumulation.
+ */
+moe_status moe_prepare_down_f16(const moe_shape* shape, const void* w_down, const void* ws_down,
+                                void* w_down_f16, void* ws_down_f16, void* ws, size_t ws_bytes,
+                                void* stream);
 
 /*
  * FP8 routed experts. Source: "Qwen3.8, weights in hand: 98% of a 2.4T model is routed

@@ -29,6 +29,7 @@ MOE_ERR_WORKSPACE_TOO_SMALL = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ERR_DEVICE_BOUNDS = 6
+MOE_ERR_DEVICE_RANGE = 7
 
 MOE_VARIANT_AUTO = 0
 MOE_VARIANT_STREAM = 1
@@ -51,7 +52,8 @@ class moe_shape(ctypes.Structure):
 
 class moe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "router_bias", "w_gate_up", "w_down",
-                                               "ws_gate_up", "ws_down", "w_shared_gate")]
+                                               "ws_gate_up", "ws_down", "w_shared_gate",
+                                               "w_down_f16", "ws_down_f16")]
 
 
 class moe_fp8_experts(ctypes.Structure):
@@ -80,6 +82,7 @@ _SIGS = {
     "moe_layer_forward": ([_SP, _vp, _WP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_layer_forward_host": ([_SP, _vp, _WP, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_quantize_fp8_experts": ([_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "moe_prepare_down_f16": ([_SP, _vp, _vp, _vp, _vp, _vp, _sz, _vp], ctypes.c_int),
     "moe_layer_forward_fp8": ([_SP, _vp, _WP, _FP, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
                               ctypes.c_int),
     "moe_ep_counts": ([_i32, _i32, _vp, _vp, _vp, _vp], ctypes.c_int),
@@ -157,7 +160,8 @@ def make_weights(w: dict) -> moe_weights:
     """moe_weights from a dict of device tensors keyed like the C struct."""
     return moe_weights(_ptr(w["w_router"]), _ptr(w.get("router_bias")), _ptr(w["w_gate_up"]),
                        _ptr(w["w_down"]), _ptr(w["ws_gate_up"]), _ptr(w["ws_down"]),
-                       _ptr(w["w_shared_gate"]))
+                       _ptr(w["w_shared_gate"]), _ptr(w.get("w_down_f16")),
+                       _ptr(w.get("ws_down_f16")))
 
 
 def make_fp8_experts(q: dict) -> moe_fp8_experts:
@@ -266,6 +270,12 @@ def moe_quantize_fp8_experts(shape, w_gate_up, w_down, q_gate_up, s_gate_up, q_d
                                          _ptr(q_gate_up), _ptr(s_gate_up), _ptr(q_down),
                                          _ptr(s_down), _stream(stream)),
            "moe_quantize_fp8_experts")
+
+
+def moe_prepare_down_f16(shape, w_down, ws_down, w_down_f16, ws_down_f16, ws=None, stream=None):
+    _check(_lib.moe_prepare_down_f16(ctypes.byref(shape), _ptr(w_down), _ptr(ws_down),
+                                     _ptr(w_down_f16), _ptr(ws_down_f16), *_ws_args(ws),
+                                     _stream(stream)), "moe_prepare_down_f16")
 
 
 def moe_layer_forward_fp8(shape, x, weights, experts, out, ws, topk_ids=None, topk_w=None,
@@ -400,3 +410,21 @@ def quantize_fp8_experts(shape: moe_shape, weights: dict, stream=None) -> dict:
     moe_quantize_fp8_experts(shape, weights["w_gate_up"], weights["w_down"], q["q_gate_up"],
                              q["s_gate_up"], q["q_down"], q["s_down"], stream)
     return q
+
+
+def prepare_down_f16(shape: moe_shape, weights: dict, stream=None) -> dict:
+    """The fp16 down-operand pre-pass on a weight dict (run once): returns a new dict with
+    w_down_f16 (fp16 [E][H][I]) and ws_down_f16 (fp16 [H][Is]) added. Raises if a weight
+    saturated."""
+    import torch
+
+    d = weights["w_down"].device
+    out = dict(weights)
+    out["w_down_f16"] = torch.empty(tuple(weights["w_down"].shape), dtype=torch.float16, device=d)
+    out["ws_down_f16"] = torch.empty(tuple(weights["ws_down"].shape), dtype=torch.float16, device=d)
+    ws = torch.zeros(256, dtype=torch.uint8, device=d)
+    moe_prepare_down_f16(shape, weights["w_down"], weights["ws_down"], out["w_down_f16"],
+                         out["ws_down_f16"], ws, stream)
+    st, flags = moe_device_status(ws, stream)
+    _check(st, "moe_prepare_down_f16 (device)")
+    return out

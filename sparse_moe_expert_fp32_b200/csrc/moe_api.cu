@@ -136,6 +136,9 @@ moe_status check_expert_weights(const moe_weights* w) {
   if (!w || !aligned16(w->w_gate_up) || !aligned16(w->w_down) || !aligned16(w->ws_gate_up) ||
       !aligned16(w->ws_down))
     return MOE_ERR_INVALID_ARG;
+  // the fp16 down operands: both or neither
+  if ((w->w_down_f16 || w->ws_down_f16) && (!aligned16(w->w_down_f16) || !aligned16(w->ws_down_f16)))
+    return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -193,9 +196,14 @@ moe_status run_grouped(const moe_shape& s, const Layout& L, char* ws, const uint
                        cudaStream_t st) {
   const int v = variant_of(ws);
   if (use_tc(s, v)) {
-    if (use_tc2_gate_up(s, v)) MOE_CUDA(launch_tc2_gate_up(s, L, ws, x, sorted_token, w, st));
-    else MOE_CUDA(launch_tc_gate_up(s, L, ws, x, sorted_token, w, st));
-    if (use_tc2_down(v))
+    // fp16 down operands given: h is stored as fp16(h 2^-8) and the down GEMM runs on CTA
+    // pairs with one MMA per K step (any tensor-core variant)
+    const int f16 = (w.w_down_f16 && w.ws_down_f16) ? 1 : 0;
+    if (use_tc2_gate_up(s, v)) MOE_CUDA(launch_tc2_gate_up(s, L, ws, x, sorted_token, w, f16, st));
+    else MOE_CUDA(launch_tc_gate_up(s, L, ws, x, sorted_token, w, f16, st));
+    if (f16)
+      MOE_CUDA(launch_tc2_down_f16(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));
+    else if (use_tc2_down(v))
       MOE_CUDA(launch_tc2_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));
     else
       MOE_CUDA(launch_tc_down(s, L, ws, sorted_token, sorted_w, sgate, w, y, y_shared, out, st));
@@ -284,6 +292,7 @@ moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const int32
     // no tile reads the shared expert's matrices; its tensor maps still need a valid base
     wv.ws_gate_up = wv.w_gate_up;
     wv.ws_down = wv.w_down;
+    if (wv.w_down_f16) wv.ws_down_f16 = wv.w_down_f16;
     s.Is = s.I;  // the workspace layout for Is = I is no larger than the caller's
   }
   MOE_TRY(check_expert_weights(&wv));
@@ -416,6 +425,25 @@ moe_status moe_compact_zero_channels(const moe_shape* shape, const void* w_gate_
                                 static_cast<const uint16_t*>(w_down), src, I_c,
                                 static_cast<uint16_t*>(gate_up_c), static_cast<uint16_t*>(down_c),
                                 st));
+  return MOE_OK;
+}
+
+moe_status moe_prepare_down_f16(const moe_shape* shape, const void* w_down, const void* ws_down,
+                                void* w_down_f16, void* ws_down_f16, void* ws, size_t ws_bytes,
+                                void* stream) {
+  MOE_TRY(check_shape(shape));
+  const moe_shape& s = *shape;
+  if (!aligned16(w_down) || !aligned16(ws_down) || !aligned16(w_down_f16) ||
+      !aligned16(ws_down_f16))
+    return MOE_ERR_INVALID_ARG;
+  if (ws && (!aligned16(ws) || ws_bytes < 256)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  const int sms = sm_count_host();
+  MOE_CUDA(launch_down_to_f16(static_cast<const uint16_t*>(w_down), (size_t)s.E * s.H * s.I,
+                              static_cast<uint16_t*>(w_down_f16), status, sms, st));
+  MOE_CUDA(launch_down_to_f16(static_cast<const uint16_t*>(ws_down), (size_t)s.H * s.Is,
+                              static_cast<uint16_t*>(ws_down_f16), status, sms, st));
   return MOE_OK;
 }
 
@@ -559,6 +587,7 @@ moe_status moe_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* 
   if (detail) *detail = flags;
   if (flags & kFlagTimeout) return MOE_ERR_DEVICE_TIMEOUT;
   if (flags & kFlagBounds) return MOE_ERR_DEVICE_BOUNDS;
+  if (flags & kFlagRange) return MOE_ERR_DEVICE_RANGE;
   return MOE_OK;
 }
 
@@ -609,6 +638,7 @@ const char* moe_status_string(moe_status status) {
     case MOE_ERR_CUDA: return "CUDA runtime or launch error";
     case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
     case MOE_ERR_DEVICE_BOUNDS: return "expert id out of range";
+    case MOE_ERR_DEVICE_RANGE: return "a value saturated to fit fp16 (down operands)";
   }
   return "unknown status";
 }

@@ -16,6 +16,7 @@ constexpr int kPermBlock = 256;  // tokens per dispatch block (one bit per token
 constexpr int kTcChunk = 256;    // max tokens (MMA N) per tensor-core tile
 constexpr uint32_t kFlagBounds = 1u;
 constexpr uint32_t kFlagTimeout = 2u;
+constexpr uint32_t kFlagRange = 4u;  // a value saturated to fit fp16 (down operands)
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -56,10 +57,11 @@ struct PlanView {
   int* active;    // [E+1] group ids with >= 1 row, ascending
   int* row0;      // [E+2]
   int* tp1;       // [E+2] tile prefix of the tensor-core gate|up GEMM
-  int* tp2;       // [E+2] tile prefix of the tensor-core down GEMM
+  int* tp2;       // [E+2] tile prefix of the tensor-core down GEMM (bf16 h pair, 128 rows)
+  int* tp3;       // [E+2] tile prefix of the down GEMM on fp16 operands (256 rows)
 };
 
-__host__ __device__ inline size_t plan_ints(int E) { return 1 + (size_t)(E + 1) + 3 * (size_t)(E + 2); }
+__host__ __device__ inline size_t plan_ints(int E) { return 1 + (size_t)(E + 1) + 4 * (size_t)(E + 2); }
 
 __host__ __device__ inline PlanView plan_view(void* base, int E) {
   int* p = static_cast<int*>(base);
@@ -69,12 +71,15 @@ __host__ __device__ inline PlanView plan_view(void* base, int E) {
   v.row0 = v.active + (E + 1);
   v.tp1 = v.row0 + (E + 2);
   v.tp2 = v.tp1 + (E + 2);
+  v.tp3 = v.tp2 + (E + 2);
   return v;
 }
 
 // Tensor-core tiling of a group with n rows into ceil(n / max) token chunks of nearly equal
-// size (multiples of 16 rows): max 256 rows for the gate|up GEMM, 128 for the down GEMM.
+// size (multiples of 16 rows): max 256 rows for the gate|up GEMM, 128 for the down GEMM on
+// the bf16 h pair (its MMA N is twice the rows), 256 for the down GEMM on fp16 operands.
 constexpr int kTcChunkDown = 128;
+constexpr int kTcChunkDownF16 = 256;
 // Rows per gate|up tile: decode-size batches (T*k < 16*E, a few rows per expert) chunk at
 // kTcChunkSmall, so that the one-CTA gate|up kernel's stages can be small and more of them
 // fit; larger batches at kTcChunk. The plan builder and both gate|up kernels call this with
@@ -147,6 +152,9 @@ cudaError_t launch_compact_banks(const moe_shape& s, const uint16_t* w_gate_up,
 // FP8 expert pre-pass (fp8_quant.cu): rows of n bf16 -> E4M3 codes and fp32 row scales.
 cudaError_t launch_quantize_fp8_rows(const uint16_t* w, size_t rows, int n, uint8_t* q,
                                      float* scale, int sms, cudaStream_t st);
+// Down-projection weights re-encoded as fp16(W * 2^8) (down_f16.cu); n a multiple of 8.
+cudaError_t launch_down_to_f16(const uint16_t* w, size_t n, uint16_t* out, uint32_t* status,
+                               int sms, cudaStream_t st);
 cudaError_t launch_wait_flag(const int32_t* flag, uint64_t timeout_ns, uint32_t* status,
                              cudaStream_t st);
 

@@ -75,28 +75,35 @@ __device__ void build_plan(const int* n_of, int E, int H, int I, int Is, int T, 
   const int uc = tc_gate_up_chunk(T, k, E);
   const int c0 = tc_nchunks(n0, uc), c1 = tc_nchunks(n1, uc);
   const int d0 = tc_nchunks(n0, kTcChunkDown), d1 = tc_nchunks(n1, kTcChunkDown);
+  const int f0 = tc_nchunks(n0, kTcChunkDownF16), f1 = tc_nchunks(n1, kTcChunkDownF16);
   const int t1a = (g <= E) ? c0 * (inter(g) / 128) : 0;
   const int t1b = has1 ? c1 * (Is / 128) : 0;
   const int t2a = (g <= E) ? d0 * (H / 256) : 0;
   const int t2b = has1 ? d1 * (H / 256) : 0;
+  const int t3a = (g <= E) ? f0 * (H / 256) : 0;
+  const int t3b = has1 ? f1 * (H / 256) : 0;
   const int r0a = (g <= E) ? n0 : 0, r0b = has1 ? n1 : 0;
-  int tot1, tot2, totr;
+  int tot1, tot2, tot3, totr;
   const int p1 = block_exclusive_scan(t1a + t1b, smem, &tot1);
   const int p2 = block_exclusive_scan(t2a + t2b, smem, &tot2);
+  const int p3 = block_exclusive_scan(t3a + t3b, smem, &tot3);
   const int pr = block_exclusive_scan(r0a + r0b, smem, &totr);
   if (g <= E) {
     pv.tp1[g] = p1;
     pv.tp2[g] = p2;
+    pv.tp3[g] = p3;
     pv.row0[g] = pr;
   }
   if (has1) {
     pv.tp1[E] = p1 + t1a;
     pv.tp2[E] = p2 + t2a;
+    pv.tp3[E] = p3 + t3a;
     pv.row0[E] = pr + r0a;
   }
   if (threadIdx.x == 0) {
     pv.tp1[E + 1] = tot1;
     pv.tp2[E + 1] = tot2;
+    pv.tp3[E + 1] = tot3;
     pv.row0[E + 1] = totr;
   }
 }

@@ -195,6 +195,11 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(const void* p) {
 }
 
 // Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major.
+// Instruction descriptor of kind::f16: fp32 accumulator, fp16 A and B, both K-major.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }

@@ -67,7 +67,10 @@ constexpr int kSlotCols = 256;
 constexpr int kBoxes = 5;  // token boxes of 128, 64, 32, 16 and 8 rows
 __host__ __device__ constexpr int box_rows(int i) { return 128 >> i; }
 
-enum PairMode { kPairGateUp = 0, kPairDown = 1 };
+// kPairDownF16: the down GEMM on fp16 operands (W' = W * 2^8 from the weight pre-pass,
+// h' = h * 2^-8 in plane 0): tiles of up to 256 rows, MMA N = rows, each CTA holding half of
+// the tile's rows; one MMA per K step where the bf16 pair needs hi and lo columns.
+enum PairMode { kPairGateUp = 0, kPairDown = 1, kPairDownF16 = 2 };
 
 struct PairShared {
   uint64_t full[kMaxStages];   // leader: both CTAs' copies of a stage have landed
@@ -131,7 +134,8 @@ __device__ __forceinline__ PairGeom pair_geom(const TcArgs& a, const PairShared&
   constexpr int kStageK = Ring<KSUB>::kStageK;
   PairGeom G;
   G.t = decode_tile(S.row0, S.tp, a.E, tile,
-                    MODE == kPairGateUp ? tc_gate_up_chunk(a.T, a.k, a.E) : kTcChunkDown);
+                    MODE == kPairGateUp ? tc_gate_up_chunk(a.T, a.k, a.E)
+                                        : (MODE == kPairDown ? kTcChunkDown : kTcChunkDownF16));
   G.shared = G.t.g == a.E;
   if (MODE == kPairGateUp) {
     const int Ig = G.shared ? a.Is : a.I;
@@ -142,13 +146,21 @@ __device__ __forceinline__ PairGeom pair_geom(const TcArgs& a, const PairShared&
     G.b_row = (G.shared ? G.t.p0 - R : G.t.p0) + rank * G.nb;
     G.n_mma = G.t.N;
     G.nk = a.H / kStageK;
-  } else {
+  } else if (MODE == kPairDown) {
     const int base = G.shared ? 0 : G.t.g * a.H;
     G.a_row0 = base + G.t.m * 256 + rank * 128;
     G.a_row1 = 0;
     G.nb = G.t.N;
     G.b_row = G.t.p0 + rank * plane_rows;
     G.n_mma = 2 * G.t.N;
+    G.nk = (G.shared ? a.Is : a.I) / kStageK;
+  } else {  // kPairDownF16: rows [0, N/2) of plane 0 in CTA 0, [N/2, N) in CTA 1
+    const int base = G.shared ? 0 : G.t.g * a.H;
+    G.a_row0 = base + G.t.m * 256 + rank * 128;
+    G.a_row1 = 0;
+    G.nb = G.t.N / 2;
+    G.b_row = G.t.p0 + rank * G.nb;
+    G.n_mma = G.t.N;
     G.nk = (G.shared ? a.Is : a.I) / kStageK;
   }
   return G;
@@ -171,7 +183,7 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   const int pair = (int)ptx::cluster_id_x(), npairs = (int)ptx::cluster_count_x();
   const int E = args.E;
   const PlanView pv = plan_view(const_cast<int*>(args.plan), E);
-  const int* tp = (MODE == kPairGateUp) ? pv.tp1 : pv.tp2;
+  const int* tp = (MODE == kPairGateUp) ? pv.tp1 : (MODE == kPairDown ? pv.tp2 : pv.tp3);
   for (int g = threadIdx.x; g < E + 2; g += blockDim.x) {
     S.tp[g] = tp[g];
     S.row0[g] = pv.row0[g];
@@ -226,7 +238,7 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         my_map = G.shared ? &tm_a_sh : &tm_a;
         my_off = lane * (kASub / 2);
         my_row = lane ? G.a_row1 : G.a_row0;
-      } else if (MODE == kPairDown && lane == 0) {
+      } else if (MODE != kPairGateUp && lane == 0) {
         my_map = G.shared ? &tm_a_sh : &tm_a;
         my_row = G.a_row0;
       } else if (lane >= 2) {
@@ -291,7 +303,8 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         }
         ptx::tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(slot * kSlotCols);
-        const uint32_t idesc = ptx::idesc_bf16_f32(256, G.n_mma);
+        const uint32_t idesc = MODE == kPairDownF16 ? ptx::idesc_f16_f32(256, G.n_mma)
+                                                    : ptx::idesc_bf16_f32(256, G.n_mma);
         for (int ks = 0; ks < G.nk; ++ks) {
           // The copies' completion on the full barrier orders them before the MMAs that
           // read the stage; no tcgen05 fence is needed here.
@@ -344,11 +357,18 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
       const uint32_t base = tmem + lane_off + (uint32_t)(slot * kSlotCols);
       // down: token and weight of this warp's columns, requested before waiting for the
       // accumulator so that the loads overlap the tile's MMAs
-      int col_tok[2] = {0, 0};
-      float col_w[2] = {0.f, 0.f};
-      if (MODE == kPairDown) {
+      // down: 32-column chunks per warp half (N <= 128 with the bf16 pair, <= 256 with fp16)
+      constexpr int kDownChunks = MODE == kPairDownF16 ? 4 : 2;
+      int col_tok[kDownChunks];
+      float col_w[kDownChunks];
 #pragma unroll
-        for (int ci = 0; ci < 2; ++ci) {
+      for (int ci = 0; ci < kDownChunks; ++ci) {
+        col_tok[ci] = 0;
+        col_w[ci] = 0.f;
+      }
+      if (MODE != kPairGateUp) {
+#pragma unroll
+        for (int ci = 0; ci < kDownChunks; ++ci) {
           const int c = (2 * ci + half) * 32 + lane;
           if (c < tl.nvalid) {
             const int p = tl.p0 + c;
@@ -385,28 +405,32 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
               if (c0 + j < tl.nvalid) {
                 const float gv = __uint_as_float(r[j]);
                 // SiLU(g) = g / (1 + e^-g) with the fast exponential and division (a few
-                // ulp; h is carried with about 16 significant bits)
+                // ulp; h is carried with 16 or, for fp16 down operands, 11 significant bits)
                 const float hv = __fdividef(gv, 1.f + __expf(-gv)) * xu[j][lane];
-                const uint16_t hi = f32_to_bf16_rn(hv);
                 const size_t at = (size_t)(tl.p0 + c0 + j) * args.ldh + ch;
-                args.h[at] = hi;
-                args.h[args.h_plane + at] = f32_to_bf16_rn(hv - bf16lo(hi));
+                store_h(args.h, args.h_plane, at, hv, args.h_f16, args.status);
               }
             }
           }
         }
       } else {
-        // columns [0, N) hold W h_hi and [N, 2N) W h_lo of the same rows
+        // bf16 pair: columns [0, N) hold W h_hi and [N, 2N) W h_lo of the same rows;
+        // fp16 operands: columns [0, N) hold W h
         const int mrow = tl.m * 256 + rank * 128 + q * 32 + 4 * (lane & 7);  // this lane's channels
         const int H = args.H;
         float4(&xpz)[8][8] = S.xpose[warp - 2];
 #pragma unroll
-        for (int ci = 0; ci < 2; ++ci) {
+        for (int ci = 0; ci < kDownChunks; ++ci) {
           const int c0 = (2 * ci + half) * 32;
           if (c0 >= tl.nvalid) break;
           uint32_t r0[32], r1[32];
           ptx::tmem_ld32(base + (uint32_t)c0, r0);
-          ptx::tmem_ld32(base + (uint32_t)(tl.N + c0), r1);
+          if (MODE == kPairDown) {
+            ptx::tmem_ld32(base + (uint32_t)(tl.N + c0), r1);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r1[j] = 0u;  // +0.0f
+          }
           ptx::tmem_ld_wait();
           // 32 channels (lanes) x 32 tokens (registers); every 8 tokens go through shared
           // memory so that eight lanes own the 32 channels (128 bytes) of one token and each
@@ -464,9 +488,10 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
 
 // ---------------------------------------------------------------- host side
 
-bool make_pair_maps(PairMaps* b, const void* base, uint64_t inner, uint64_t outer) {
+bool make_pair_maps(PairMaps* b, const void* base, uint64_t inner, uint64_t outer,
+                    CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   for (int i = 0; i < kBoxes; ++i)
-    if (!make_map(&b->m[i], base, inner, outer, kBK, (uint32_t)box_rows(i))) return false;
+    if (!make_map(&b->m[i], base, inner, outer, kBK, (uint32_t)box_rows(i), dt)) return false;
   return true;
 }
 
@@ -514,7 +539,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& a_sh, const Pai
 }  // namespace
 
 cudaError_t launch_tc2_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
-                               const int32_t* sorted_token, const moe_weights& w,
+                               const int32_t* sorted_token, const moe_weights& w, int h_f16,
                                cudaStream_t st) {
   uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
   cudaError_t e = launch_gather_rows(s, L, ws, x, sorted_token, st);
@@ -528,6 +553,7 @@ cudaError_t launch_tc2_gate_up(const moe_shape& s, const Layout& L, char* ws, co
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
+  args.h_f16 = h_f16;
   LaunchScope scope(MOE_K_GATE_UP, st);
   return launch_pair<kPairGateUp, 2>(a, a_sh, b, b_sh, args, st);
 }
@@ -557,6 +583,30 @@ cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
   if ((s.I >= 1024 && s.Is >= 1024) || (int64_t)s.T * s.k < 16 * (int64_t)s.E)
     return launch_pair<kPairDown, 2>(a, a_sh, b, b, args, st);
   return launch_pair<kPairDown, 1>(a, a_sh, b, b, args, st);
+}
+
+cudaError_t launch_tc2_down_f16(const moe_shape& s, const Layout& L, char* ws,
+                                const int32_t* sorted_token, const float* sorted_w,
+                                const float* sgate, const moe_weights& w, float* y,
+                                float* y_shared, float* out, cudaStream_t st) {
+  CUtensorMap a, a_sh;
+  PairMaps b;
+  if (!make_map(&a, w.w_down_f16, s.I, (uint64_t)s.E * s.H, kBK, 128,
+                CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_map(&a_sh, w.ws_down_f16, s.Is, (uint64_t)s.H, kBK, 128,
+                CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_pair_maps(&b, ws + L.h, L.ldh, L.h_plane / L.ldh,  // plane 0: h' = fp16(h 2^-8)
+                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return cudaErrorInvalidValue;
+  TcArgs args = base_args(s, L, ws);
+  args.sorted_token = sorted_token;
+  args.sorted_w = sorted_w;
+  args.sgate = sgate;
+  args.y = y;
+  args.y_shared = y_shared;
+  args.out = out;
+  LaunchScope scope(MOE_K_DOWN, st);
+  return launch_pair<kPairDownF16, 2>(a, a_sh, b, b, args, st);
 }
 
 }  // namespace moe

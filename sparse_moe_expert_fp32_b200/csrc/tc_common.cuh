@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
 
 #include <mutex>
 
@@ -34,6 +35,7 @@ struct TcArgs {
   int ntiles;         // router: tile count (no plan)
   int* counter;       // next tile to hand out (zeroed before the launch)
   int* counter_next;  // gate|up: the down kernel's counter, zeroed here for its launch
+  int h_f16;          // gate|up: store h as fp16(h * 2^-8) in plane 0 (fp16 down operands)
 };
 
 struct Tile {
@@ -102,6 +104,26 @@ __device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// h = SiLU(gate) * up for the down GEMM: the bf16 pair (hi = bf16(h) at h[at], lo =
+// bf16(h - hi) at h[plane + at], about 16 significant bits) or, when the down operands are
+// fp16, h' = fp16(h * 2^-8) at h[at] (11 significant bits down to |h| = 2^-6; W' = W * 2^8
+// makes W' h' = W h). A value beyond fp16's range saturates and raises the range flag.
+__device__ __forceinline__ void store_h(uint16_t* h, size_t plane, size_t at, float hv, int f16,
+                                        uint32_t* status) {
+  if (f16) {
+    float v = hv * 0.00390625f;  // 2^-8, exact
+    if (fabsf(v) > 65504.f) {
+      v = copysignf(65504.f, v);
+      set_flag(status, kFlagRange);
+    }
+    h[at] = __half_as_ushort(__float2half_rn(v));
+  } else {
+    const uint16_t hi = f32_to_bf16_rn(hv);
+    h[at] = hi;
+    h[plane + at] = f32_to_bf16_rn(hv - bf16lo(hi));
+  }
+}
+
 __device__ __forceinline__ int token_of_row(const TcArgs& a, int p, int R) {
   if (p >= R) return p - R;
   const int t = a.sorted_token[p];
@@ -128,10 +150,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer][inner] (inner contiguous), box [box_outer][box_inner] with the
-// swizzle matching box_inner (64 elements: 128-byte swizzle, 32: 64-byte swizzle).
+// 2-D tensor of 2-byte elements [outer][inner] (inner contiguous; bf16 unless `dt` says
+// fp16), box [box_outer][box_inner] with the swizzle matching box_inner (64 elements:
+// 128-byte swizzle, 32: 64-byte swizzle).
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -140,7 +164,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
   cuuint32_t estr[2] = {1, 1};
   const CUtensorMapSwizzle sw =
       box_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

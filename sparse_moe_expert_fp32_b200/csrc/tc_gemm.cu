@@ -485,12 +485,10 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             if (c0 + j < tl.nvalid) {
               const float gv = __uint_as_float(r0[j]);
               // SiLU(g) = g / (1 + e^-g) with the fast exponential and division (a few ulp;
-              // h is carried with about 16 significant bits)
+              // h is carried with 16 or, for fp16 down operands, 11 significant bits)
               const float hv = __fdividef(gv, 1.f + __expf(-gv)) * __uint_as_float(r1[j]);
-              const uint16_t hi = f32_to_bf16_rn(hv);
               const size_t at = (size_t)(tl.p0 + c0 + j) * args.ldh + ch;
-              args.h[at] = hi;
-              args.h[args.h_plane + at] = f32_to_bf16_rn(hv - bf16lo(hi));
+              store_h(args.h, args.h_plane, at, hv, args.h_f16, args.status);
             }
           }
         } else if (MODE == kRouter) {
@@ -680,7 +678,8 @@ cudaError_t launch_gather_rows(const moe_shape& s, const Layout& L, char* ws, co
 }
 
 cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
-                              const int32_t* sorted_token, const moe_weights& w, cudaStream_t st) {
+                              const int32_t* sorted_token, const moe_weights& w, int h_f16,
+                              cudaStream_t st) {
   using C = Cfg<kGateUp>;  // kBK and box shapes are the same for kGateUpSmall
   uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
   {
@@ -698,6 +697,7 @@ cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, con
   args.sorted_token = sorted_token;
   args.counter = reinterpret_cast<int*>(ws + L.sched) + 0;
   args.counter_next = reinterpret_cast<int*>(ws + L.sched) + 1;
+  args.h_f16 = h_f16;
   LaunchScope scope(MOE_K_GATE_UP, st);
   if (tc_gate_up_chunk(s.T, s.k, s.E) == kTcChunkSmall)
     return launch_mode<kGateUpSmall>(a, a_sh, b, b_sh, args, sm_count(), st);

@@ -14,7 +14,8 @@ cudaError_t launch_tc_router(const moe_shape& s, const Layout& L, char* ws, cons
                              const float* wr, float* logits, cudaStream_t st);
 
 cudaError_t launch_tc_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
-                              const int32_t* sorted_token, const moe_weights& w, cudaStream_t st);
+                              const int32_t* sorted_token, const moe_weights& w, int h_f16,
+                              cudaStream_t st);
 cudaError_t launch_tc_down(const moe_shape& s, const Layout& L, char* ws,
                            const int32_t* sorted_token, const float* sorted_w, const float* sgate,
                            const moe_weights& w, float* y, float* y_shared, float* out,
@@ -28,11 +29,18 @@ cudaError_t launch_gather_rows(const moe_shape& s, const Layout& L, char* ws, co
 // half of a token tile, and the down GEMM takes the hi and lo halves of h in one MMA.
 // For batches with many tokens per expert (prefill).
 cudaError_t launch_tc2_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
-                               const int32_t* sorted_token, const moe_weights& w, cudaStream_t st);
+                               const int32_t* sorted_token, const moe_weights& w, int h_f16,
+                               cudaStream_t st);
 cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
                             const int32_t* sorted_token, const float* sorted_w, const float* sgate,
                             const moe_weights& w, float* y, float* y_shared, float* out,
                             cudaStream_t st);
+// The down GEMM on fp16 operands (w.w_down_f16, w.ws_down_f16 and h' = fp16(h 2^-8) in plane
+// 0 of h, written by a gate|up launch with h_f16 = 1): 256-row tiles, one MMA per K step.
+cudaError_t launch_tc2_down_f16(const moe_shape& s, const Layout& L, char* ws,
+                                const int32_t* sorted_token, const float* sorted_w,
+                                const float* sgate, const moe_weights& w, float* y,
+                                float* y_shared, float* out, cudaStream_t st);
 
 // The same grouped GEMMs with the routed experts' weights in FP8 (E4M3 codes, one fp32 scale
 // per weight row; the shared expert stays bf16): one CTA per tile, codes widened to bf16 in

@@ -127,3 +127,11 @@ def test_error_stats_leave_out_differing_id_sets():
     assert e["sample_id_sets_differ"] == 1 and e["sample_near_ties_fp64"] == 1
     assert e["max_abs_over_rms"] == pytest.approx(0.01 / rms)
     assert e["mean_rel"] == pytest.approx(0.01 / 6.0)
+
+
+def test_fp16_down_operands_bytes_by_hand():
+    # with the fp16 down operands h is one fp16 value per element: 2 bytes instead of 4
+    cfg = synth.CONFIGS["flash_decode"]
+    h2 = (640 * 640 + 64 * 640) * 2
+    assert bench.algorithmic_bytes("gate_up", cfg, 370, h_bytes=2) == 2433515520 - h2
+    assert bench.algorithmic_bytes("down", cfg, 370, h_bytes=2) == 1218150400 - h2

@@ -92,6 +92,15 @@ def _chosen_experts(st):
     return sorted(set([hot, cold, ragged] + others))
 
 
+def _weights(st, variant):
+    """The device weights, with the fp16 down operands for the *_f16 variants (made once)."""
+    if not variant.endswith("_f16"):
+        return st["dev"]
+    if "dev_f16" not in st:
+        st["dev_f16"] = moe.prepare_down_f16(moe.shape_of(st["cfg"]), st["dev"])
+    return st["dev_f16"]
+
+
 def _staged_expect(st):
     """Oracle y rows (first 64 and last tiles of chosen experts), y_shared rows (first and
     last shared tiles) and the layer on a few tokens; computed once per workload."""
@@ -125,13 +134,13 @@ def _dev(a, dtype):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name,variant", [(n, v) for n in FULL for v in ("tc", "tc2", "auto")])
+@pytest.mark.parametrize("name,variant", [(n, v) for n in FULL for v in ("tc", "tc2", "auto", "auto_f16")])
 def test_staged_entry_points_full_size(name, variant):
     st = _state(name)
-    cfg, dev = st["cfg"], st["dev"]
+    cfg, dev = st["cfg"], _weights(st, variant)
     exp = _staged_expect(st)
     s = moe.shape_of(cfg)
-    ws = moe.alloc_workspace(s, variant=VARIANTS[variant])
+    ws = moe.alloc_workspace(s, variant=VARIANTS[variant.replace("_f16", "")])
     R, T, H = cfg.R, cfg.T, cfg.H
     off = torch.empty(cfg.E + 1, dtype=torch.int32, device="cuda")
     stok = torch.empty(R, dtype=torch.int32, device="cuda")
@@ -200,13 +209,14 @@ def _layer_expect(st):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name,variant", [(n, v) for n in FULL for v in ("auto", "tc2", "tc", "stream")])
+@pytest.mark.parametrize("name,variant", [(n, v) for n in FULL
+                                          for v in ("auto", "auto_f16", "tc2", "tc", "stream")])
 def test_layer_forward_full_size_sampled(name, variant):
     st = _state(name)
-    cfg, dev = st["cfg"], st["dev"]
+    cfg, dev = st["cfg"], _weights(st, variant)
     exp = _layer_expect(st)
     s = moe.shape_of(cfg)
-    ws = moe.alloc_workspace(s, variant=VARIANTS[variant])
+    ws = moe.alloc_workspace(s, variant=VARIANTS[variant.replace("_f16", "")])
     out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
     ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device="cuda")
     moe.moe_layer_forward(s, dev["x"], dev, out, ws, topk_ids=ids)
