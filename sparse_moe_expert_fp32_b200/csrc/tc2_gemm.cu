@@ -64,8 +64,15 @@ struct Ring {
 };
 constexpr int kMaxStages = 6;
 constexpr int kSlotCols = 256;
-constexpr int kBoxes = 5;  // token boxes of 128, 64, 32, 16 and 8 rows
-__host__ __device__ constexpr int box_rows(int i) { return 128 >> i; }
+// Each operand of a stage arrives in one TMA instruction (measured: an instruction costs
+// the issuing thread ~90 cycles whatever its size, and the time from a freed stage to its
+// last copy request lies on the pipeline's critical path). Weights: one 5-D (gate|up: K,
+// channel row, gate/up, K block, expert) or 3-D (down: K, row, K block) box. Token rows:
+// one 3-D box (K, row, K block) whose height is the CTA's row count rounded up to 16 (the
+// rows past it are neighbours' or zero fill, and no MMA reads them): 8 tensor maps.
+constexpr int kBHeights = 8;
+__host__ __device__ constexpr int box_h(int i) { return 16 * (i + 1); }
+__device__ __forceinline__ int box_index(int nb) { return (nb + 15) / 16 - 1; }
 
 // kPairDownF16: the down GEMM on fp16 operands (W' = W * 2^8 from the weight pre-pass,
 // h' = h * 2^-8 in plane 0): tiles of up to 256 rows, MMA N = rows, each CTA holding half of
@@ -96,33 +103,17 @@ static_assert(pair_smem_bytes<1>() <= 232448 && pair_smem_bytes<2>() <= 232448,
               "over the 227 KB of shared memory a CTA may use");
 
 struct PairMaps {
-  CUtensorMap m[kBoxes];
+  CUtensorMap m[kBHeights];  // token boxes of 16, 32, ..., 128 rows
 };
-
-// This CTA's token half of an nb-row B operand as boxes of 128/64/32/16/8 rows: piece j's
-// first row and box index; false past the last piece (nb is a multiple of 8, at most 128).
-__device__ __forceinline__ bool b_piece(int nb, int j, int& row, int& bidx) {
-  int r = 0;
-#pragma unroll
-  for (int i = 0; i < kBoxes; ++i) {
-    if (nb & box_rows(i)) {
-      if (j == 0) {
-        row = r;
-        bidx = i;
-        return true;
-      }
-      --j;
-      r += box_rows(i);
-    }
-  }
-  return false;
-}
 
 struct PairGeom {
   Tile t;
-  int a_row0, a_row1;  // gate|up: the 64 gate and 64 up rows; down: 128 rows from a_row0
+  int a_row0;          // gate|up: first of the 64 channels within the gate (and up) half;
+                       // down: first of the 128 weight rows
+  int a_e;             // gate|up: expert of the 5-D weight box (0 for the shared expert)
   int b_row;           // first row of this CTA's token half in its tensor map
   int nb;              // rows of this CTA's token half
+  int nbb;             // rows of its token box (nb rounded up to 16)
   int n_mma;           // MMA N
   int nk;              // K stages
   bool shared;
@@ -138,30 +129,31 @@ __device__ __forceinline__ PairGeom pair_geom(const TcArgs& a, const PairShared&
                                         : (MODE == kPairDown ? kTcChunkDown : kTcChunkDownF16));
   G.shared = G.t.g == a.E;
   if (MODE == kPairGateUp) {
-    const int Ig = G.shared ? a.Is : a.I;
-    const int base = G.shared ? 0 : G.t.g * 2 * a.I;
-    G.a_row0 = base + G.t.m * 128 + rank * 64;
-    G.a_row1 = G.a_row0 + Ig;
+    G.a_row0 = G.t.m * 128 + rank * 64;
+    G.a_e = G.shared ? 0 : G.t.g;
     G.nb = G.t.N / 2;
     G.b_row = (G.shared ? G.t.p0 - R : G.t.p0) + rank * G.nb;
     G.n_mma = G.t.N;
     G.nk = a.H / kStageK;
+    G.nbb = (G.nb + 15) & ~15;
   } else if (MODE == kPairDown) {
     const int base = G.shared ? 0 : G.t.g * a.H;
     G.a_row0 = base + G.t.m * 256 + rank * 128;
-    G.a_row1 = 0;
+    G.a_e = 0;
     G.nb = G.t.N;
     G.b_row = G.t.p0 + rank * plane_rows;
     G.n_mma = 2 * G.t.N;
     G.nk = (G.shared ? a.Is : a.I) / kStageK;
+    G.nbb = (G.nb + 15) & ~15;
   } else {  // kPairDownF16: rows [0, N/2) of plane 0 in CTA 0, [N/2, N) in CTA 1
     const int base = G.shared ? 0 : G.t.g * a.H;
     G.a_row0 = base + G.t.m * 256 + rank * 128;
-    G.a_row1 = 0;
+    G.a_e = 0;
     G.nb = G.t.N / 2;
     G.b_row = G.t.p0 + rank * G.nb;
     G.n_mma = G.t.N;
     G.nk = (G.shared ? a.Is : a.I) / kStageK;
+    G.nbb = (G.nb + 15) & ~15;
   }
   return G;
 }
@@ -206,7 +198,7 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tm_a);
     ptx::prefetch_tmap(&tm_a_sh);
-    for (int i = 0; i < kBoxes; ++i) {
+    for (int i = 0; i < kBHeights; ++i) {
       ptx::prefetch_tmap(&tm_b.m[i]);
       ptx::prefetch_tmap(&tm_b_sh.m[i]);
     }
@@ -224,33 +216,17 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     // Lane 0 waits for this CTA's copy of a stage to be free (and in the leader arms the
-    // full barrier with both CTAs' bytes); then each lane with a box issues it: lanes 0-1
-    // the weight rows, lanes 2.. the pieces of this CTA's token half.
+    // full barrier with both CTAs' bytes); then lane 0 issues the weight box and lane 1 the
+    // box of this CTA's token rows, each covering all KSUB K blocks of the stage.
     const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(&S.full[0]), 0);
     int it = 0;
     bool aborted = false;
     for (int tile = pair; tile < total && !aborted; tile += npairs) {
       const PairGeom G = pair_geom<MODE, KSUB>(args, S, tile, R, rank, plane_rows);
-      const CUtensorMap* my_map = nullptr;
-      uint32_t my_off = 0;
-      int my_row = 0;
-      if (MODE == kPairGateUp && lane < 2) {  // 64 gate rows, then 64 up rows
-        my_map = G.shared ? &tm_a_sh : &tm_a;
-        my_off = lane * (kASub / 2);
-        my_row = lane ? G.a_row1 : G.a_row0;
-      } else if (MODE != kPairGateUp && lane == 0) {
-        my_map = G.shared ? &tm_a_sh : &tm_a;
-        my_row = G.a_row0;
-      } else if (lane >= 2) {
-        int r, bi;
-        if (b_piece(G.nb, lane - 2, r, bi)) {
-          const PairMaps& bm = (MODE == kPairGateUp && G.shared) ? tm_b_sh : tm_b;
-          my_map = &bm.m[bi];
-          my_off = kABytes + (uint32_t)r * kRowB;  // sub-tile j adds j * kBSub
-          my_row = G.b_row + r;
-        }
-      }
-      const uint32_t bytes = 2u * KSUB * (kASub + (uint32_t)G.nb * kRowB);  // both CTAs
+      const CUtensorMap* a_map = G.shared ? &tm_a_sh : &tm_a;
+      const CUtensorMap* b_map =
+          &((MODE == kPairGateUp && G.shared) ? tm_b_sh : tm_b).m[box_index(G.nb)];
+      const uint32_t bytes = 2u * KSUB * (kASub + (uint32_t)G.nbb * kRowB);  // both CTAs
       for (int ks = 0; ks < G.nk; ++ks, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -263,12 +239,16 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           aborted = true;
           break;
         }
-        if (my_map)
-#pragma unroll
-          for (int j = 0; j < KSUB; ++j)  // weight sub-tiles at j * kASub, token ones at j * kBSub
-            ptx::tma_load_2d_pair(smem + s * kStageBytes + my_off + j * (my_off < kABytes ? kASub : kBSub),
-                                  my_map, full0 + (uint32_t)(s * sizeof(uint64_t)),
-                                  ks * kStageK + j * kBK, my_row);
+        uint8_t* st = smem + s * kStageBytes;
+        const uint32_t bar = full0 + (uint32_t)(s * sizeof(uint64_t));
+        if (lane == 0) {
+          if (MODE == kPairGateUp)  // [K block][gate, up][64 channels][64 K]
+            ptx::tma_load_5d_pair(st, a_map, bar, 0, G.a_row0, 0, ks * KSUB, G.a_e);
+          else  // [K block][128 rows][64 K]
+            ptx::tma_load_3d_pair(st, a_map, bar, 0, G.a_row0, ks * KSUB);
+        } else if (lane == 1) {  // [K block][nbb token rows][64 K]
+          ptx::tma_load_3d_pair(st + kABytes, b_map, bar, 0, G.b_row, ks * KSUB);
+        }
       }
     }
     // wait until the MMAs have released every stage this CTA filled, so that no commit
@@ -319,7 +299,7 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           if (KSUB == 2) {
             ptx::umma_bf16_pair_x4(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
             ready = ptx::mbar_test_wait(&S.full[s2], ph2);
-            ptx::umma_bf16_pair_x4(d, ad + (kASub >> 4), bd + (kBSub >> 4), idesc, 1u);
+            ptx::umma_bf16_pair_x4(d, ad + (kASub >> 4), bd + ((G.nbb * kRowB) >> 4), idesc, 1u);
           } else {
             ptx::umma_bf16_pair_x2(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
             ready = ptx::mbar_test_wait(&S.full[s2], ph2);
@@ -488,11 +468,36 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
 
 // ---------------------------------------------------------------- host side
 
-bool make_pair_maps(PairMaps* b, const void* base, uint64_t inner, uint64_t outer,
-                    CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
-  for (int i = 0; i < kBoxes; ++i)
-    if (!make_map(&b->m[i], base, inner, outer, kBK, (uint32_t)box_rows(i), dt)) return false;
+// Token rows [rows][ld] (2-byte elements) as 3-D boxes {64 K, h rows, KSUB K blocks} for the
+// eight box heights.
+template <int KSUB>
+bool make_token_maps(PairMaps* b, const void* base, uint64_t ld, uint64_t rows,
+                     CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  const uint64_t dims[3] = {(uint64_t)kBK, rows, ld / kBK};
+  const uint64_t strides[2] = {ld * 2, kRowB};
+  for (int i = 0; i < kBHeights; ++i) {
+    const uint32_t box[3] = {(uint32_t)kBK, (uint32_t)box_h(i), (uint32_t)KSUB};
+    if (!make_map_nd(&b->m[i], base, 3, dims, strides, box, dt)) return false;
+  }
   return true;
+}
+
+// Gate|up weights [E][2I][H] as 5-D boxes {64 K, 64 channels, gate and up, KSUB K blocks, 1}.
+bool make_gate_up_map(CUtensorMap* m, const void* base, uint64_t E, uint64_t I, uint64_t H) {
+  const uint64_t dims[5] = {(uint64_t)kBK, I, 2, H / kBK, E};
+  const uint64_t strides[4] = {H * 2, I * H * 2, kRowB, 2 * I * H * 2};
+  const uint32_t box[5] = {(uint32_t)kBK, 64, 2, 2, 1};
+  return make_map_nd(m, base, 5, dims, strides, box);
+}
+
+// Down weights [rows][I] as 3-D boxes {64 K, 128 rows, KSUB K blocks}.
+template <int KSUB>
+bool make_down_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t I,
+                   CUtensorMapDataType dt) {
+  const uint64_t dims[3] = {(uint64_t)kBK, rows, I / kBK};
+  const uint64_t strides[2] = {I * 2, kRowB};
+  const uint32_t box[3] = {(uint32_t)kBK, 128, (uint32_t)KSUB};
+  return make_map_nd(m, base, 3, dims, strides, box, dt);
 }
 
 template <int MODE, int KSUB>
@@ -546,10 +551,10 @@ cudaError_t launch_tc2_gate_up(const moe_shape& s, const Layout& L, char* ws, co
   if (e != cudaSuccess) return e;
   CUtensorMap a, a_sh;
   PairMaps b, b_sh;
-  if (!make_map(&a, w.w_gate_up, s.H, (uint64_t)s.E * 2 * s.I, kBK, 64) ||
-      !make_map(&a_sh, w.ws_gate_up, s.H, 2ull * s.Is, kBK, 64) ||
-      !make_pair_maps(&b, xs, s.H, (uint64_t)s.T * s.k) ||
-      !make_pair_maps(&b_sh, x, s.H, (uint64_t)s.T))
+  if (!make_gate_up_map(&a, w.w_gate_up, s.E, s.I, s.H) ||
+      !make_gate_up_map(&a_sh, w.ws_gate_up, 1, s.Is, s.H) ||
+      !make_token_maps<2>(&b, xs, s.H, (uint64_t)s.T * s.k) ||
+      !make_token_maps<2>(&b_sh, x, s.H, (uint64_t)s.T))
     return cudaErrorInvalidValue;
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
@@ -558,16 +563,22 @@ cudaError_t launch_tc2_gate_up(const moe_shape& s, const Layout& L, char* ws, co
   return launch_pair<kPairGateUp, 2>(a, a_sh, b, b_sh, args, st);
 }
 
-cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
-                            const int32_t* sorted_token, const float* sorted_w, const float* sgate,
-                            const moe_weights& w, float* y, float* y_shared, float* out,
-                            cudaStream_t st) {
+template <int MODE, int KSUB>
+cudaError_t launch_down_mode(const moe_shape& s, const Layout& L, char* ws, const void* wd,
+                             const void* wsd, CUtensorMapDataType dt, const TcArgs& args,
+                             cudaStream_t st) {
   CUtensorMap a, a_sh;
   PairMaps b;
-  if (!make_map(&a, w.w_down, s.I, (uint64_t)s.E * s.H, kBK, 128) ||
-      !make_map(&a_sh, w.ws_down, s.Is, (uint64_t)s.H, kBK, 128) ||
-      !make_pair_maps(&b, ws + L.h, L.ldh, 2 * (L.h_plane / L.ldh)))
+  const uint64_t rows = (MODE == kPairDown ? 2 : 1) * (L.h_plane / L.ldh);  // h planes used
+  if (!make_down_map<KSUB>(&a, wd, (uint64_t)s.E * s.H, s.I, dt) ||
+      !make_down_map<KSUB>(&a_sh, wsd, (uint64_t)s.H, s.Is, dt) ||
+      !make_token_maps<KSUB>(&b, ws + L.h, L.ldh, rows, dt))
     return cudaErrorInvalidValue;
+  return launch_pair<MODE, KSUB>(a, a_sh, b, b, args, st);
+}
+
+TcArgs down_args(const moe_shape& s, const Layout& L, char* ws, const int32_t* sorted_token,
+                 const float* sorted_w, const float* sgate, float* y, float* y_shared, float* out) {
   TcArgs args = base_args(s, L, ws);
   args.sorted_token = sorted_token;
   args.sorted_w = sorted_w;
@@ -575,38 +586,33 @@ cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
   args.y = y;
   args.y_shared = y_shared;
   args.out = out;
+  return args;
+}
+
+cudaError_t launch_tc2_down(const moe_shape& s, const Layout& L, char* ws,
+                            const int32_t* sorted_token, const float* sorted_w, const float* sgate,
+                            const moe_weights& w, float* y, float* y_shared, float* out,
+                            cudaStream_t st) {
+  const TcArgs args = down_args(s, L, ws, sorted_token, sorted_w, sgate, y, y_shared, out);
   LaunchScope scope(MOE_K_DOWN, st);
   // 128-K stages (eight MMAs per producer/issuer hand-off) for long down loops (I >= 1024)
   // and for decode-size batches, whose tiny MMAs (N = 2 x a few rows) leave the issuing
   // thread as the bound with the copies landing far ahead; 64-K stages and a 6-deep ring
   // for short loops at prefill sizes (inter 640: 5 stages per tile)
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if ((s.I >= 1024 && s.Is >= 1024) || (int64_t)s.T * s.k < 16 * (int64_t)s.E)
-    return launch_pair<kPairDown, 2>(a, a_sh, b, b, args, st);
-  return launch_pair<kPairDown, 1>(a, a_sh, b, b, args, st);
+    return launch_down_mode<kPairDown, 2>(s, L, ws, w.w_down, w.ws_down, bf, args, st);
+  return launch_down_mode<kPairDown, 1>(s, L, ws, w.w_down, w.ws_down, bf, args, st);
 }
 
 cudaError_t launch_tc2_down_f16(const moe_shape& s, const Layout& L, char* ws,
                                 const int32_t* sorted_token, const float* sorted_w,
                                 const float* sgate, const moe_weights& w, float* y,
                                 float* y_shared, float* out, cudaStream_t st) {
-  CUtensorMap a, a_sh;
-  PairMaps b;
-  if (!make_map(&a, w.w_down_f16, s.I, (uint64_t)s.E * s.H, kBK, 128,
-                CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_map(&a_sh, w.ws_down_f16, s.Is, (uint64_t)s.H, kBK, 128,
-                CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_pair_maps(&b, ws + L.h, L.ldh, L.h_plane / L.ldh,  // plane 0: h' = fp16(h 2^-8)
-                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
-    return cudaErrorInvalidValue;
-  TcArgs args = base_args(s, L, ws);
-  args.sorted_token = sorted_token;
-  args.sorted_w = sorted_w;
-  args.sgate = sgate;
-  args.y = y;
-  args.y_shared = y_shared;
-  args.out = out;
+  const TcArgs args = down_args(s, L, ws, sorted_token, sorted_w, sgate, y, y_shared, out);
   LaunchScope scope(MOE_K_DOWN, st);
-  return launch_pair<kPairDownF16, 2>(a, a_sh, b, b, args, st);
+  return launch_down_mode<kPairDownF16, 2>(s, L, ws, w.w_down_f16, w.ws_down_f16,
+                                           CU_TENSOR_MAP_DATA_TYPE_FLOAT16, args, st);
 }
 
 }  // namespace moe

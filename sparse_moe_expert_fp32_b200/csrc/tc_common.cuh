@@ -169,6 +169,26 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// n-D tensor of 2-byte elements (bf16 unless `dt` says fp16): dims innermost first,
+// strides (bytes) of dims 1..n-1, box per dim; the 128-byte swizzle (64-element rows).
+bool make_map_nd(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides, const uint32_t* box,
+                 CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  auto fn = encode_fn();
+  if (!fn || rank < 2 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  return fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), d, st, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   cudaGetDevice(&dev);

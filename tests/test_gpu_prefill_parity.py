@@ -35,7 +35,8 @@ from parity_util import assert_layer_close, id_sets_match  # noqa: E402
 VARIANTS = {"stream": moe.MOE_VARIANT_STREAM, "tc": moe.MOE_VARIANT_TC,
             "tc2": moe.MOE_VARIANT_TC2, "auto": moe.MOE_VARIANT_AUTO}
 FULL = ["flash_prefill", "t24_prefill", "t24_skewed"]
-GATE_UP_TILE, DOWN_TILE = 256, 128
+# rows per tile: gate|up; down with h as the bf16 pair; down on fp16 operands
+GATE_UP_TILE, DOWN_TILE, DOWN_TILE_F16 = 256, 128, 256
 
 
 def _chunks(n, max_rows):
@@ -47,7 +48,7 @@ def _chunks(n, max_rows):
 
 def _last_tile_rows(n):
     """Row range [a, n) covering the last gate|up tile and the last down tile of a group."""
-    a = min(_chunks(n, GATE_UP_TILE)[-1][0], _chunks(n, DOWN_TILE)[-1][0])
+    a = min(_chunks(n, m)[-1][0] for m in (GATE_UP_TILE, DOWN_TILE, DOWN_TILE_F16))
     return a, n
 
 
@@ -242,7 +243,10 @@ def test_tile_split_matches_the_kernels_plan():
             ch = _chunks(n, m)
             assert sum(r for _, r in ch) == n and all(r > 0 for _, r in ch)
             assert all(a % 16 == 0 for a, _ in ch) and max(r for _, r in ch) <= m
-    assert _last_tile_rows(210) == (128, 210) and _last_tile_rows(100) == (0, 100)
+    assert _chunks(210, DOWN_TILE) == [(0, 112), (112, 98)]
+    assert _chunks(600, GATE_UP_TILE) == [(0, 208), (208, 208), (416, 184)]
+    assert _last_tile_rows(210) == (0, 210) and _last_tile_rows(600) == (416, 600)
+    assert _last_tile_rows(12131) == (12032, 12131)
 
 
 # ----------------------------------------------------------------------------- router ties
