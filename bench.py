@@ -51,6 +51,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCES = {  # kernel id -> source file whose hash a stored ncu traffic figure carries
     "gate_up": ("stream_swiglu.cu", "tc_gemm.cu", "tc2_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
     "down": ("stream_swiglu.cu", "tc_gemm.cu", "tc2_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
+    "gate_up_f16": ("tc_gemm.cu", "tc2_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
+    "down_f16": ("tc2_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
     "router_logits": ("router.cu", "tc_gemm.cu", "tc_common.cuh", "sm100_ptx.cuh"),
     "router_topk": ("router.cu",),
     "permute": ("permute.cu",),
