@@ -145,9 +145,9 @@ def algorithmic_bytes(kernel: str, cfg, n_active: int, fp8: bool = False, h_byte
     with the fp16 down operands)."""
     T, H, I, Is, R = cfg.T, cfg.H, cfg.I, cfg.Is, cfg.R
     if fp8 and kernel == "gate_up":
-        return n_active * 2 * I * (H + 4) + (2 * Is * H + T * H) * 2 + (R * I + T * Is) * 4
+        return n_active * 2 * I * (H + 4) + (2 * Is * H + T * H) * 2 + (R * I + T * Is) * h_bytes
     if fp8 and kernel == "down":
-        return n_active * H * (I + 4) + H * Is * 2 + (R * I + T * Is) * 4 + T * H * 4
+        return n_active * H * (I + 4) + H * Is * 2 + (R * I + T * Is) * h_bytes + T * H * 4
     if kernel == "gate_up":  # activated experts' gate|up + shared gate|up + x + h out
         return (n_active * 2 * I * H + 2 * Is * H + T * H) * 2 + (R * I + T * Is) * h_bytes
     if kernel == "down":  # activated experts' down + shared down + h in + out (fp32)
@@ -438,9 +438,10 @@ def measure_workload(args, cfg, world, rank, local, sampler, want_cpu_baseline: 
         torch.cuda.empty_cache()
         qs = moe.make_fp8_experts(q)
     down_f16 = None
-    if fp8 is None and not args.down_bf16_pair and args.variant != "stream":
+    if not args.down_bf16_pair and (fp8 is not None or args.variant != "stream"):
         # weight pre-pass (once, at load time): the down matrices re-encoded as fp16(W * 2^8)
-        # so that the down GEMM takes h as one fp16 value (one MMA per K step)
+        # so that the down GEMM takes h as one fp16 value (one MMA per K step); with the FP8
+        # experts only the shared expert's matrix (the routed codes widen to fp16 exactly)
         t0 = time.time()
         dev = moe.prepare_down_f16(s, dev)
         torch.cuda.synchronize()
@@ -712,9 +713,9 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
             "us_per_layer": head["us_per_layer"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": ("e4m3 (gate|up MMAs), bf16 (down MMAs)" if args.fp8 else
-                      "bf16 (router split, gate|up MMAs)" + ("" if head.get("down_operands_fp16") is None
-                                                             else ", fp16 (down MMAs)")
+            "dtype": (("e4m3 (gate|up MMAs)" if args.fp8 else "bf16 (router split, gate|up MMAs)")
+                      + (", bf16 (down MMAs)" if head.get("down_operands_fp16") is None
+                         else ", fp16 (down MMAs)")
                       + ", fp32 accumulation and output"),
             "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random "
                     "router; the skewed layer adds a Zipf(1.1) router bias and 71% zero gate/up channels)"}

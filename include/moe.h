@@ -309,8 +309,9 @@ moe_status moe_compact_zero_channels(const moe_shape* shape, const void* w_gate_
  * saturate and set the range flag. An intermediate |h| above 65504 * 2^8 saturates and sets
  * the range flag too (moe_device_status: MOE_ERR_DEVICE_RANGE).
  * moe_prepare_down_f16: w_down bf16 [E][H][I] -> w_down_f16 fp16 [E][H][I]; ws_down bf16
- *   [H][Is] -> ws_down_f16 fp16 [H][Is]; asynchronous on `stream`. ws (optional, may be
- *   NULL) receives the range flag in its status word.
+ *   [H][Is] -> ws_down_f16 fp16 [H][Is]; asynchronous on `stream`. w_down and w_down_f16
+ *   may both be NULL (only the shared expert's matrix is re-encoded: what the FP8 layer
+ *   uses). ws (optional, may be NULL) receives the range flag in its status word.
  * Pass the results as moe_weights.w_down_f16 / ws_down_f16: moe_layer_forward,
  * moe_layer_forward_host and moe_grouped_swiglu then use them whenever they take the
  * tensor-core kernels (the down GEMM then runs on CTA pairs); the weight-streaming variant
@@ -339,7 +340,10 @@ moe_status moe_prepare_down_f16(const moe_shape* shape, const void* w_down, cons
  *   [E][2I][H] and w_down [E][H][I] -> the four arrays above; asynchronous on `stream`.
  *   Errors: MOE_ERR_INVALID_ARG (null or misaligned pointer), MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA.
  * moe_layer_forward_fp8: moe_layer_forward with the routed experts taken from `experts`
- *   (weights->w_gate_up and weights->w_down are not read and may be NULL). Supported for
+ *   (weights->w_gate_up and weights->w_down are not read and may be NULL). With
+ *   weights->ws_down_f16 given (moe_prepare_down_f16), h is carried as one fp16 value and
+ *   the codes are widened to fp16 for the down GEMM (one MMA per K step, deeper staging);
+ *   without it, as the bf16 pair. Supported for
  *   decode-size batches, T*k < 16*E, with I and Is multiples of 128 and H of 256 on
  *   sm_100; otherwise MOE_ERR_UNSUPPORTED. Same outputs, workspace and errors as
  *   moe_layer_forward.

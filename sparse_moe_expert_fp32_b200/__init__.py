@@ -414,17 +414,19 @@ def quantize_fp8_experts(shape: moe_shape, weights: dict, stream=None) -> dict:
 
 def prepare_down_f16(shape: moe_shape, weights: dict, stream=None) -> dict:
     """The fp16 down-operand pre-pass on a weight dict (run once): returns a new dict with
-    w_down_f16 (fp16 [E][H][I]) and ws_down_f16 (fp16 [H][Is]) added. Raises if a weight
-    saturated."""
+    w_down_f16 (fp16 [E][H][I]; None when the dict has no routed w_down) and ws_down_f16
+    (fp16 [H][Is]) added. Raises if a weight saturated."""
     import torch
 
-    d = weights["w_down"].device
+    d = weights["ws_down"].device
     out = dict(weights)
-    out["w_down_f16"] = torch.empty(tuple(weights["w_down"].shape), dtype=torch.float16, device=d)
+    routed = weights.get("w_down") is not None  # absent: only the shared expert (FP8 layer)
+    out["w_down_f16"] = (torch.empty(tuple(weights["w_down"].shape), dtype=torch.float16, device=d)
+                         if routed else None)
     out["ws_down_f16"] = torch.empty(tuple(weights["ws_down"].shape), dtype=torch.float16, device=d)
     ws = torch.zeros(256, dtype=torch.uint8, device=d)
-    moe_prepare_down_f16(shape, weights["w_down"], weights["ws_down"], out["w_down_f16"],
-                         out["ws_down_f16"], ws, stream)
+    moe_prepare_down_f16(shape, weights["w_down"] if routed else None, weights["ws_down"],
+                         out["w_down_f16"], out["ws_down_f16"], ws, stream)
     st, flags = moe_device_status(ws, stream)
     _check(st, "moe_prepare_down_f16 (device)")
     return out

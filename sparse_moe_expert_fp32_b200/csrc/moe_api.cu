@@ -2,6 +2,8 @@
 // variant choice and the order of kernel launches for each stage of the layer
 // (Qwen3.8-Flash-Next architecture study, MoE pipeline "Router -> Top 10 + normalize ->
 // Dispatch R tokens -> Grouped expert GEMMs -> Weighted combine + gated shared expert").
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <mutex>
 #include <unordered_map>
@@ -82,8 +84,16 @@ cudaEvent_t pool_event() {
 
 }  // namespace
 
+// NVTX range names per moe_kernel id (host ranges around each launch: they show the layer's
+// stages on a profiler's timeline and cost a few nanoseconds when no tool is attached)
+const char* const kKernelNames[MOE_K_COUNT] = {"moe.router_logits", "moe.router_topk",
+                                               "moe.permute",       "moe.gate_up",
+                                               "moe.down",          "moe.combine",
+                                               "moe.other"};
+
 LaunchScope::LaunchScope(moe_kernel id, cudaStream_t s, int nkernels) : slot(-1), stream(s) {
   g_launches.fetch_add((uint64_t)nkernels, std::memory_order_relaxed);
+  nvtxRangePushA(kKernelNames[(int)id < MOE_K_COUNT ? (int)id : MOE_K_OTHER]);
   if (!g_prof_on) return;
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
@@ -97,6 +107,7 @@ LaunchScope::LaunchScope(moe_kernel id, cudaStream_t s, int nkernels) : slot(-1)
 }
 
 LaunchScope::~LaunchScope() {
+  nvtxRangePop();
   if (slot < 0) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (slot < (int)g_recs.size()) cudaEventRecord(g_recs[slot].b, stream);
@@ -433,15 +444,18 @@ moe_status moe_prepare_down_f16(const moe_shape* shape, const void* w_down, cons
                                 void* stream) {
   MOE_TRY(check_shape(shape));
   const moe_shape& s = *shape;
-  if (!aligned16(w_down) || !aligned16(ws_down) || !aligned16(w_down_f16) ||
+  // the routed pair may be left out (both NULL): the FP8 layer needs only the shared one
+  const bool routed = w_down || w_down_f16;
+  if ((routed && (!aligned16(w_down) || !aligned16(w_down_f16))) || !aligned16(ws_down) ||
       !aligned16(ws_down_f16))
     return MOE_ERR_INVALID_ARG;
   if (ws && (!aligned16(ws) || ws_bytes < 256)) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   uint32_t* status = static_cast<uint32_t*>(ws);
   const int sms = sm_count_host();
-  MOE_CUDA(launch_down_to_f16(static_cast<const uint16_t*>(w_down), (size_t)s.E * s.H * s.I,
-                              static_cast<uint16_t*>(w_down_f16), status, sms, st));
+  if (routed)
+    MOE_CUDA(launch_down_to_f16(static_cast<const uint16_t*>(w_down), (size_t)s.E * s.H * s.I,
+                                static_cast<uint16_t*>(w_down_f16), status, sms, st));
   MOE_CUDA(launch_down_to_f16(static_cast<const uint16_t*>(ws_down), (size_t)s.H * s.Is,
                               static_cast<uint16_t*>(ws_down_f16), status, sms, st));
   return MOE_OK;
@@ -475,6 +489,7 @@ moe_status moe_layer_forward_fp8(const moe_shape* shape, const void* x, const mo
   const moe_shape& s = *shape;
   MOE_TRY(check_router_weights(weights));
   if (!aligned16(weights->ws_gate_up) || !aligned16(weights->ws_down)) return MOE_ERR_INVALID_ARG;
+  if (weights->ws_down_f16 && !aligned16(weights->ws_down_f16)) return MOE_ERR_INVALID_ARG;
   if (!experts || !aligned16(experts->q_gate_up) || !aligned16(experts->s_gate_up) ||
       !aligned16(experts->q_down) || !aligned16(experts->s_down))
     return MOE_ERR_INVALID_ARG;

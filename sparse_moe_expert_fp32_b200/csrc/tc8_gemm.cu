@@ -7,10 +7,13 @@
 // weight instead of two, which is what bounds a decode-size batch. Two kernels, one CTA per
 // tile, swap AB as in the bf16 kernels (2 x 128 weight rows on the MMA's M side, tokens on N):
 //
-// down (tc8_down_kernel): weight-only. The E4M3 codes are widened to bf16 in shared memory
-// (exactly: a code has a 4-bit significand) and the tensor cores run the bf16 MMAs of the
-// bf16 layer on h's hi and lo rows (one MMA of N = 2 x rows, up to 128 rows), K = 64 per
-// stage. Roles of the 320 threads:
+// down (tc8_down_kernel): weight-only. The E4M3 codes are widened in shared memory
+// (exactly: a code has a 4-bit significand) and the tensor cores run the MMAs of the bf16
+// layer, K = 64 per stage. Two forms (template F16): widened to bf16 against h's hi and lo
+// rows (one MMA of N = 2 x rows, up to 128 rows); or, when the fp16 down operands are given
+// (the shared expert's fp16(W x 2^8) and h' = fp16(h x 2^-8)), widened to fp16 against the
+// one h' plane (N = rows), which halves the h rows a staging slot holds, so four slots fit
+// where three did. Roles of the 320 threads:
 //   warp 0      TMA producer over a ring of staging slots: per stage, the E4M3 codes of
 //               the 256 weight rows (16 KB, plain 64-byte rows) and the h rows;
 //   warp 1      TMEM owner and MMA issuer (lane 0);
@@ -49,20 +52,22 @@ constexpr uint32_t kAccBytes = 128 * kRowB;    // 128 weight rows of bf16: one a
 constexpr uint32_t kQRowB = 64;                // one E4M3 row of a stage
 constexpr uint32_t kQBytes = 256 * kQRowB;     // 256 weight rows of E4M3 (= kAccBytes)
 constexpr int kBoxHeights8 = 4;                // token boxes of 128, 64, 32, 16 rows
-constexpr int kARing = 2;                      // bf16 operand slots
+constexpr int kARing = 2;                      // widened operand slots
+constexpr int kMaxSlots8 = 4;
 
+template <bool F16>
 struct Cfg8 {
   static constexpr int kMaxTile = kTcChunkDown;
-  static constexpr int kBTiles = 2;  // hi and lo rows of h
+  static constexpr int kBTiles = F16 ? 1 : 2;  // h' rows, or hi and lo rows of h
   static constexpr uint32_t kBBytes = (uint32_t)kBTiles * kMaxTile * kRowB;
   static constexpr uint32_t kSlotBytes = kQBytes + kBBytes;  // a multiple of 1024
-  static constexpr int kSlots = 3;
+  static constexpr int kSlots = F16 ? 4 : 3;
   static constexpr uint32_t kAStage = 2 * kAccBytes;
 };
 
 struct Shared8 {
-  uint64_t sfull[Cfg8::kSlots];
-  uint64_t sempty[Cfg8::kSlots];
+  uint64_t sfull[kMaxSlots8];
+  uint64_t sempty[kMaxSlots8];
   uint64_t aready[kARing];
   uint64_t afree[kARing];
   uint64_t tmem_full[2];
@@ -78,13 +83,16 @@ struct Shared8 {
   float4 xpose[kEpiWarps8][8][8];  // down epilogue: per warp, 8 tokens x 32 channels
 };
 
+template <bool F16>
 constexpr size_t smem8_bytes() {
-  using C = Cfg8;
+  using C = Cfg8<F16>;
   return 1024 + (size_t)C::kSlots * C::kSlotBytes + (size_t)kARing * C::kAStage + sizeof(Shared8);
 }
-static_assert(smem8_bytes() <= 232448, "over the 227 KB of shared memory a CTA may use");
-static_assert(Cfg8::kSlotBytes % 1024 == 0,
+static_assert(smem8_bytes<false>() <= 232448 && smem8_bytes<true>() <= 232448,
+              "over the 227 KB of shared memory a CTA may use");
+static_assert(Cfg8<false>::kSlotBytes % 1024 == 0 && Cfg8<true>::kSlotBytes % 1024 == 0,
               "staging slots must keep 1024-byte alignment for the 128-byte swizzle");
+static_assert(Cfg8<true>::kSlots <= kMaxSlots8 && Cfg8<false>::kSlots <= kMaxSlots8, "slots");
 
 struct TokenMaps8 {
   CUtensorMap m[kBoxHeights8];
@@ -137,7 +145,7 @@ __device__ __forceinline__ Geom8 geom8(const TcArgs& a, const Shared8& S, int ti
   const int nsh = total - tpE;
   const int t2 = tile < nsh ? tpE + tile : tile - nsh;
   Geom8 G;
-  G.t = decode_tile(S.row0, S.tp, a.E, t2, Cfg8::kMaxTile);
+  G.t = decode_tile(S.row0, S.tp, a.E, t2, Cfg8<false>::kMaxTile);
   G.shared = G.t.g == a.E;
   const int base = G.shared ? 0 : G.t.g * a.H;
   G.a_row0 = base + G.t.m * 256;
@@ -180,10 +188,29 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w) {
   return r;
 }
 
+// The same to two fp16. Shifting left by 7 and masking leaves sign | 0 | exponent(4) |
+// mantissa(3) << 7, the fp16 pattern of code * 2^-8 (fp16's exponent bias is 8 above E4M3's;
+// E4M3 subnormals become fp16 subnormals with the same relation); the fp16 multiply by 2^8
+// gives the code's value, exact (at most 4 significant bits, at most 448).
+template <uint32_t kSel>
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
+  uint32_t t, r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(w), "r"(0u), "r"(kSel));
+  t = (t << 7) & 0xBF80BF80u;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(t), "r"(0x5C005C00u), "r"(0x80008000u));
+  return r;
+}
+
+template <bool F16, uint32_t kSel>
+__device__ __forceinline__ uint32_t widen8(uint32_t w) {
+  return F16 ? e4m3x2_to_f16x2<kSel>(w) : e4m3x2_to_bf16x2<kSel>(w);
+}
+
+template <bool F16>
 __global__ void __launch_bounds__(kThreads8, 1)
 tc8_down_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_a_sh,
                 const __grid_constant__ TokenMaps8 tm_b, const Tc8Args a8) {
-  using C = Cfg8;
+  using C = Cfg8<F16>;
   const TcArgs& args = a8.a;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -329,8 +356,9 @@ tc8_down_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::mbar_arrive(&S.q_empty[slot]);
         if (tile < 0) break;
         const Geom8 G = geom8(args, S, tile, total, R);
-        const int cols = 2 * G.t.N;  // columns [0, N) W h_hi, [N, 2N) W h_lo
-        const uint32_t idesc = ptx::idesc_bf16_f32(128, cols);
+        // bf16: columns [0, N) W h_hi, [N, 2N) W h_lo; fp16: columns [0, N) W h'
+        const int cols = F16 ? G.t.N : 2 * G.t.N;
+        const uint32_t idesc = F16 ? ptx::idesc_f16_f32(128, cols) : ptx::idesc_bf16_f32(128, cols);
         int first, count;
         sl.take(cols, first, count);
         for (int i = 0; i < count && !aborted; ++i) {
@@ -394,7 +422,7 @@ tc8_down_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (tile < 0) break;
       const Geom8 G = geom8(args, S, tile, total, R);
       if (G.shared) {
-        js += G.nk;  // bf16 weights: nothing to widen
+        js += G.nk;  // 16-bit weights: nothing to widen
         continue;
       }
       bool ok = true;
@@ -416,10 +444,10 @@ tc8_down_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const int q = i * (32 * kConvWarps) + ct;
           const int row = q >> 2, ch = q & 3;
           const uint4 v = *reinterpret_cast<const uint4*>(src + row * kQRowB + ch * 16);
-          const uint4 o0 = make_uint4(e4m3x2_to_bf16x2<0x9180>(v.x), e4m3x2_to_bf16x2<0xB3A2>(v.x),
-                                      e4m3x2_to_bf16x2<0x9180>(v.y), e4m3x2_to_bf16x2<0xB3A2>(v.y));
-          const uint4 o1 = make_uint4(e4m3x2_to_bf16x2<0x9180>(v.z), e4m3x2_to_bf16x2<0xB3A2>(v.z),
-                                      e4m3x2_to_bf16x2<0x9180>(v.w), e4m3x2_to_bf16x2<0xB3A2>(v.w));
+          const uint4 o0 = make_uint4(widen8<F16, 0x9180>(v.x), widen8<F16, 0xB3A2>(v.x),
+                                      widen8<F16, 0x9180>(v.y), widen8<F16, 0xB3A2>(v.y));
+          const uint4 o1 = make_uint4(widen8<F16, 0x9180>(v.z), widen8<F16, 0xB3A2>(v.z),
+                                      widen8<F16, 0x9180>(v.w), widen8<F16, 0xB3A2>(v.w));
           const int r = row & 127;
           uint8_t* base = dst + (row >> 7) * kAccBytes + r * kRowB;
           *reinterpret_cast<uint4*>(base + (((2 * ch) ^ (r & 7)) << 4)) = o0;
@@ -436,7 +464,7 @@ tc8_down_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int ew = warp - 2 - kConvWarps;  // 0 .. kEpiWarps8 - 1
     const int qd = warp & 3;               // TMEM lanes 32*qd .. +31 (warp % 4 rule)
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    constexpr int kChunks = Cfg8::kMaxTile / 32;
+    constexpr int kChunks = Cfg8<F16>::kMaxTile / 32;
     Slots8 sl;
     for (int qi = 0;; ++qi) {
       const int slot = qi % kQueue8;
@@ -449,7 +477,7 @@ tc8_down_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const Geom8 G = geom8(args, S, tile, total, R);
       const Tile& tl = G.t;
       int first, count;
-      sl.take(2 * tl.N, first, count);
+      sl.take(F16 ? tl.N : 2 * tl.N, first, count);
       const uint32_t b0 = tmem + lane_off + first * kSlotCols8;
       const uint32_t b1 = b0 + (count == 2 ? kSlotCols8 : 128u);
       // row scales of this lane's two accumulator rows (1 for the bf16 shared expert), and
@@ -458,9 +486,10 @@ tc8_down_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       int col_tok[kChunks];
       float col_w[kChunks];
       if (!G.shared) {
+        // fp16 operands: h' = h 2^-8, so the row scale takes the 2^8 back
         const float* s = a8.scale + (size_t)tl.g * args.H + tl.m * 256 + qd * 32 + lane;
-        sc0 = __ldg(s);
-        sc1 = __ldg(s + 128);
+        sc0 = __ldg(s) * (F16 ? 256.f : 1.f);
+        sc1 = __ldg(s + 128) * (F16 ? 256.f : 1.f);
       }
 #pragma unroll
       for (int ci = 0; ci < kChunks; ++ci) {
@@ -487,15 +516,24 @@ tc8_down_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t r0[32], r1[32];
         ptx::tmem_ld32(b0 + c0, r0);
         ptx::tmem_ld32(b1 + c0, r1);
-        // lo half of h in columns N + c0 (inside the accumulator's region: N <= 128)
-        uint32_t l0[32], l1[32];
-        ptx::tmem_ld32(b0 + tl.N + c0, l0);
-        ptx::tmem_ld32(b1 + tl.N + c0, l1);
-        ptx::tmem_ld_wait();
+        if (!F16) {
+          // lo half of h in columns N + c0 (inside the accumulator's region: N <= 128)
+          uint32_t l0[32], l1[32];
+          ptx::tmem_ld32(b0 + tl.N + c0, l0);
+          ptx::tmem_ld32(b1 + tl.N + c0, l1);
+          ptx::tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          r0[j] = __float_as_uint((__uint_as_float(r0[j]) + __uint_as_float(l0[j])) * sc0);
-          r1[j] = __float_as_uint((__uint_as_float(r1[j]) + __uint_as_float(l1[j])) * sc1);
+          for (int j = 0; j < 32; ++j) {
+            r0[j] = __float_as_uint((__uint_as_float(r0[j]) + __uint_as_float(l0[j])) * sc0);
+            r1[j] = __float_as_uint((__uint_as_float(r1[j]) + __uint_as_float(l1[j])) * sc1);
+          }
+        } else {
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            r0[j] = __float_as_uint(__uint_as_float(r0[j]) * sc0);
+            r1[j] = __float_as_uint(__uint_as_float(r1[j]) * sc1);
+          }
         }
         {
           // 32 channels (lanes) x 32 tokens (registers) per accumulator, regrouped through
@@ -891,12 +929,11 @@ tc8_gate_up_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int j = 0; j < 32; ++j) {
           if (c0 + j < tl.nvalid) {
             const float gv = __uint_as_float(r0[j]);
-            // SiLU(g) = g / (1 + e^-g), fast exponential and division (h carries ~16 bits)
+            // SiLU(g) = g / (1 + e^-g), fast exponential and division (h carries 16 or,
+            // for fp16 down operands, 11 significant bits)
             const float hv = __fdividef(gv, 1.f + __expf(-gv)) * __uint_as_float(r1[j]);
-            const uint16_t hi = f32_to_bf16_rn(hv);
             const size_t at = (size_t)(tl.p0 + c0 + j) * args.ldh + ch;
-            args.h[at] = hi;
-            args.h[args.h_plane + at] = f32_to_bf16_rn(hv - bf16lo(hi));
+            store_h(args.h, args.h_plane, at, hv, args.h_f16, args.status);
           }
         }
       }
@@ -1010,16 +1047,18 @@ bool make_token_maps8(TokenMaps8* b, const void* base, uint64_t inner, uint64_t 
   return true;
 }
 
+template <bool F16>
 cudaError_t launch8_down(const CUtensorMap& q, const CUtensorMap& a_sh, const TokenMaps8& b,
                          const Tc8Args& args, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(tc8_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)smem8_bytes());
+    attr_err = cudaFuncSetAttribute(tc8_down_kernel<F16>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem8_bytes<F16>());
   });
   if (attr_err != cudaSuccess) return attr_err;
-  tc8_down_kernel<<<sm_count(), kThreads8, smem8_bytes(), st>>>(q, a_sh, b, args);
+  tc8_down_kernel<F16><<<sm_count(), kThreads8, smem8_bytes<F16>(), st>>>(q, a_sh, b, args);
   return cudaGetLastError();
 }
 
@@ -1061,6 +1100,7 @@ cudaError_t launch_tc8_gate_up(const moe_shape& s, const Layout& L, char* ws, co
   args.a.counter_next = reinterpret_cast<int*>(ws + L.sched) + 1;
   args.scale = q.s_gate_up;
   args.x_scale = x_scale;
+  args.a.h_f16 = w.ws_down_f16 ? 1 : 0;  // fp16 down operands: h as fp16(h 2^-8)
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -1079,8 +1119,10 @@ cudaError_t launch_tc8_down(const moe_shape& s, const Layout& L, char* ws,
                             float* y_shared, float* out, cudaStream_t st) {
   CUtensorMap qm, a_sh;
   TokenMaps8 b;
+  const bool f16 = w.ws_down_f16 != nullptr;  // then the gate|up kernel stored h as fp16
   if (!make_map_e4m3(&qm, q.q_down, s.I, (uint64_t)s.E * s.H) ||
-      !make_map(&a_sh, w.ws_down, s.Is, (uint64_t)s.H, kBK8, 128) ||
+      !make_map(&a_sh, f16 ? w.ws_down_f16 : w.ws_down, s.Is, (uint64_t)s.H, kBK8, 128,
+                f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
       !make_token_maps8(&b, ws + L.h, L.ldh, 2 * (L.h_plane / L.ldh)))
     return cudaErrorInvalidValue;
   Tc8Args args{};
@@ -1094,7 +1136,7 @@ cudaError_t launch_tc8_down(const moe_shape& s, const Layout& L, char* ws,
   args.a.counter = reinterpret_cast<int*>(ws + L.sched) + 1;
   args.scale = q.s_down;
   LaunchScope scope(MOE_K_DOWN, st);
-  return launch8_down(qm, a_sh, b, args, st);
+  return f16 ? launch8_down<true>(qm, a_sh, b, args, st) : launch8_down<false>(qm, a_sh, b, args, st);
 }
 
 }  // namespace moe

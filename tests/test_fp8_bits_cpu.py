@@ -1,9 +1,10 @@
 """CPU checks of the two bit-level identities the FP8 kernels rely on (no GPU).
 
 1. The down kernel widens E4M3 codes to bf16 with prmt (selectors and mask read from the
-   kernel source), a shift, a mask and one bf16 multiply by 2^120. Emulated here for all
-   65536 code pairs and both selectors, it must give every finite code's exact value
-   (PyTorch's float8_e4m3fn decoder), subnormals and signed zeros included.
+   kernel source), a shift, a mask and one bf16 multiply by 2^120, or to fp16 with a shift
+   by 7, another mask and one fp16 multiply by 2^8. Emulated here for all 65536 code pairs
+   and both selectors, both must give every finite code's exact value (PyTorch's
+   float8_e4m3fn decoder), subnormals and signed zeros included.
 2. The gate|up kernel carries a bf16 token row as two E4M3 pieces with a power-of-two row
    scale 2^k (amax 2^k in [128, 256)). Emulated with PyTorch's round-to-nearest-even E4M3
    conversion: x 2^k = hi + lo exactly for every element within 2^9 of the row's largest
@@ -39,13 +40,18 @@ def _bf16_to_f64(u16: np.ndarray) -> np.ndarray:
 
 def test_widening_constants_give_exact_values():
     src = open(SRC).read()
-    sels = sorted(set(int(m, 16) for m in re.findall(r"e4m3x2_to_bf16x2<(0x[0-9A-Fa-f]+)>", src)))
+    sels = sorted(set(int(m, 16) for m in re.findall(r"widen8<F16, (0x[0-9A-Fa-f]+)>", src)))
     assert sels == [0x9180, 0xB3A2], sels
     mask = int(re.search(r"\(t << 4\) & (0x[0-9A-Fa-f]+)u", src).group(1), 16)
     mul = int(re.search(r'"r"\((0x[0-9A-Fa-f]+)u\), "r"\(0x80008000u\)', src).group(1), 16)
     assert mul & 0xFFFF == mul >> 16
     factor = _bf16_to_f64(np.array([mul & 0xFFFF], np.uint16))[0]
     assert factor == 2.0 ** 120
+    # the fp16 form: shift 7, its mask, and an fp16 multiply by 2^8
+    mask16 = int(re.search(r"\(t << 7\) & (0x[0-9A-Fa-f]+)u", src).group(1), 16)
+    mul16 = int(re.search(r'fma\.rn\.f16x2.*?"r"\((0x[0-9A-Fa-f]+)u\), "r"\(0x80008000u\)', src).group(1), 16)
+    assert mul16 & 0xFFFF == mul16 >> 16
+    assert np.array([mul16 & 0xFFFF], np.uint16).view(np.float16)[0] == 256.0
 
     pairs = np.arange(1 << 16, dtype=np.uint32)
     ref = torch.from_numpy(np.arange(256, dtype=np.uint8)).view(torch.float8_e4m3fn).double().numpy()
@@ -54,6 +60,14 @@ def test_widening_constants_give_exact_values():
         t = (_prmt(w, sel) << 4) & mask
         for half, codes in ((t & 0xFFFF, pairs & 0xFF), (t >> 16, pairs >> 8)):
             got = _bf16_to_f64(half.astype(np.uint16)) * factor  # exact in fp64
+            want = ref[codes]
+            fin = ~np.isnan(want)
+            assert np.array_equal(got[fin], want[fin])
+            assert np.array_equal(np.signbit(got[fin]), np.signbit(want[fin]))
+        t16 = (_prmt(w, sel) << 7) & mask16
+        for half, codes in ((t16 & 0xFFFF, pairs & 0xFF), (t16 >> 16, pairs >> 8)):
+            f16 = half.astype(np.uint16).view(np.float16)
+            got = (f16 * np.float16(256.0)).astype(np.float64)  # the fp16 multiply (RNE)
             want = ref[codes]
             fin = ~np.isnan(want)
             assert np.array_equal(got[fin], want[fin])

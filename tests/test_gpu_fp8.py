@@ -52,7 +52,9 @@ def _quantize(cfg, dev):
     return q
 
 
-def _forward_fp8(cfg, dev, q):
+def _forward_fp8(cfg, dev, q, f16=False):
+    """The FP8 layer; with f16, on the fp16 down operands (the shared expert's matrix
+    re-encoded, h as one fp16 value, codes widened to fp16)."""
     s = moe.shape_of(cfg)
     ws = moe.alloc_workspace(s)
     out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
@@ -60,6 +62,8 @@ def _forward_fp8(cfg, dev, q):
     w = dict(dev)
     w["w_gate_up"] = None  # the FP8 layer does not read the bf16 routed banks
     w["w_down"] = None
+    if f16:
+        w = moe.prepare_down_f16(s, w)
     moe.moe_layer_forward_fp8(s, dev["x"], w, q, out, ws, topk_ids=ids)
     st, flags = moe.moe_device_status(ws)
     assert st == moe.MOE_OK, (st, flags)
@@ -107,21 +111,23 @@ def test_quantize_bitexact_flash_decode_experts():
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("f16", [False, True])
 @pytest.mark.parametrize("case", sorted(CASES))
-def test_fp8_layer_small(case):
+def test_fp8_layer_small(case, f16):
     cfg = TINY.replace(name=case, **CASES[case])
     assert cfg.T * cfg.k < 16 * cfg.E
     dev = synth.device_inputs(cfg, seed=4)
     host = synth.host_inputs(cfg, seed=4)
     q = _quantize(cfg, dev)
-    out, ids = _forward_fp8(cfg, dev, q)
+    out, ids = _forward_fp8(cfg, dev, q, f16)
     fp8 = oracle.Fp8Experts(host.gate_up, host.down)
     stats, ties = _check(cfg, host, fp8, out, ids, list(range(cfg.T)))
-    print(case, stats, "near-ties", ties)
+    print(case, f16, stats, "near-ties", ties)
 
 
 @pytest.mark.gpu
-def test_fp8_layer_hot_expert_several_tiles():
+@pytest.mark.parametrize("f16", [False, True])
+def test_fp8_layer_hot_expert_several_tiles(f16):
     """Every token on expert 7: 200 routed rows in one group (four 64-row gate|up tiles, two
     112-row down tiles that take both TMEM slots) and 200 shared rows."""
     cfg = TINY.replace(name="hot_decode", T=200, E=256, k=4)
@@ -133,14 +139,15 @@ def test_fp8_layer_hot_expert_several_tiles():
     host = synth.host_inputs(cfg, seed=8)
     host.router_bias = bias
     q = _quantize(cfg, dev)
-    out, ids = _forward_fp8(cfg, dev, q)
+    out, ids = _forward_fp8(cfg, dev, q, f16)
     assert (ids == 7).any(axis=1).all()
     fp8 = oracle.Fp8Experts(host.gate_up, host.down)
     _check(cfg, host, fp8, out, ids, list(range(cfg.T)))
 
 
 @pytest.mark.gpu
-def test_fp8_layer_subnormal_codes():
+@pytest.mark.parametrize("f16", [False, True])
+def test_fp8_layer_subnormal_codes(f16):
     """Every routed weight row gets one outlier (640) in column 0, so its scale is 640/448
     and nearly all its other codes are E4M3 subnormals (|w / scale| < 2^-6). Column 0 of x
     is zeroed and gate row 0 of every expert too (h_0 = 0), so the outliers add nothing and
@@ -161,19 +168,20 @@ def test_fp8_layer_subnormal_codes():
     q = _quantize(cfg, dev)
     codes = q["q_gate_up"][:, 1:, 1:].cpu().numpy()
     assert ((codes & 0x78) == 0).mean() > 0.5  # most codes are subnormal (or zero)
-    out, ids = _forward_fp8(cfg, dev, q)
+    out, ids = _forward_fp8(cfg, dev, q, f16)
     fp8 = oracle.Fp8Experts(lambda e: gu[e], lambda e: dn[e])
     stats, _ = _check(cfg, host, fp8, out, ids, list(range(cfg.T)))
     print("subnormal", stats)
 
 
 @pytest.mark.gpu
-def test_fp8_layer_flash_decode_sampled():
+@pytest.mark.parametrize("f16", [False, True])
+def test_fp8_layer_flash_decode_sampled(f16):
     """The Flash-Next decode layer at full size (T=64, E=512, k=10, I=640), as timed."""
     cfg = synth.CONFIGS["flash_decode"]
     dev = synth.device_inputs(cfg, seed=0)
     q = _quantize(cfg, dev)
-    out, ids = _forward_fp8(cfg, dev, q)
+    out, ids = _forward_fp8(cfg, dev, q, f16)
     del dev, q
     torch.cuda.empty_cache()
     host = synth.host_inputs(cfg, seed=0)
