@@ -438,10 +438,10 @@ def measure_workload(args, cfg, world, rank, local, sampler, want_cpu_baseline: 
         torch.cuda.empty_cache()
         qs = moe.make_fp8_experts(q)
     down_f16 = None
-    if not args.down_bf16_pair and (fp8 is not None or args.variant != "stream"):
+    if fp8 is None and not args.down_bf16_pair and args.variant != "stream":
         # weight pre-pass (once, at load time): the down matrices re-encoded as fp16(W * 2^8)
-        # so that the down GEMM takes h as one fp16 value (one MMA per K step); with the FP8
-        # experts only the shared expert's matrix (the routed codes widen to fp16 exactly)
+        # so that the down GEMM takes h as one fp16 value (one MMA per K step). Not with the
+        # FP8 experts: their down GEMM takes h as four E4M3 pieces (16 bits)
         t0 = time.time()
         dev = moe.prepare_down_f16(s, dev)
         torch.cuda.synchronize()
@@ -635,7 +635,8 @@ def measure_workload(args, cfg, world, rank, local, sampler, want_cpu_baseline: 
 
 
 HEADLINE = "t24_prefill"
-SUITE = ("t24_prefill", "flash_decode", "flash_prefill", "t24_skewed")
+# "+fp8": the same workload with the routed experts in FP8 (as --fp8)
+SUITE = ("t24_prefill", "flash_decode", "flash_prefill", "t24_skewed", "flash_decode+fp8")
 # tokens the oracle evaluates per workload for the error statistics (and the CPU baseline)
 ERROR_SAMPLE = {"tiny": 64, "flash_decode": 16, "flash_prefill": 16, "flash_prefill_e64": 16,
                 "flash_decode_e64": 16, "t24_prefill_e16": 4, "t24_prefill": 4, "t24_skewed": 4}
@@ -675,11 +676,13 @@ def main():
     if args.no_oracle:
         args.no_cpu_baseline = True
     names = [args.workload] if args.workload else list(SUITE)
+    if args.workload is None and (args.fp8 or args.compact or args.staged):
+        names = [n for n in names if "+" not in n]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
-        line = run_reference(args, synth.CONFIGS[names[0]], world, rank)
+        line = run_reference(args, synth.CONFIGS[names[0].split("+")[0]], world, rank)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
@@ -696,9 +699,16 @@ def main():
     results = []
     try:
         for i, name in enumerate(names):
-            results.append(measure_workload(args, synth.CONFIGS[name], world, rank, local, sampler,
-                                            want_cpu_baseline=(i == 0 and world == 1
-                                                               and not args.no_cpu_baseline)))
+            base, _, extra = name.partition("+")
+            wargs = argparse.Namespace(**vars(args))
+            if extra == "fp8":
+                wargs.fp8 = True
+            r = measure_workload(wargs, synth.CONFIGS[base], world, rank, local, sampler,
+                                 want_cpu_baseline=(i == 0 and world == 1
+                                                    and not args.no_cpu_baseline))
+            if extra:
+                r["workload"] = name
+            results.append(r)
     finally:
         if sampler:
             sampler.stop()
@@ -713,9 +723,10 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
             "us_per_layer": head["us_per_layer"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": (("e4m3 (gate|up MMAs)" if args.fp8 else "bf16 (router split, gate|up MMAs)")
-                      + (", bf16 (down MMAs)" if head.get("down_operands_fp16") is None
-                         else ", fp16 (down MMAs)")
+            "dtype": ("e4m3 (routed gate|up and down MMAs: x as 2, h as 4 E4M3 pieces), bf16 (shared "
+                      "expert), fp32 accumulation and output" if args.fp8 else
+                      "bf16 (router split, gate|up MMAs)" + (", bf16 (down MMAs)" if head.get(
+                          "down_operands_fp16") is None else ", fp16 (down MMAs)")
                       + ", fp32 accumulation and output"),
             "data": "synthetic (seeded counter-based generator: x~N(0,1), weights~N(0,0.02), random "
                     "router; the skewed layer adds a Zipf(1.1) router bias and 71% zero gate/up channels)"}

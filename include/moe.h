@@ -310,8 +310,8 @@ moe_status moe_compact_zero_channels(const moe_shape* shape, const void* w_gate_
  * the range flag too (moe_device_status: MOE_ERR_DEVICE_RANGE).
  * moe_prepare_down_f16: w_down bf16 [E][H][I] -> w_down_f16 fp16 [E][H][I]; ws_down bf16
  *   [H][Is] -> ws_down_f16 fp16 [H][Is]; asynchronous on `stream`. w_down and w_down_f16
- *   may both be NULL (only the shared expert's matrix is re-encoded: what the FP8 layer
- *   uses). ws (optional, may be NULL) receives the range flag in its status word.
+ *   may both be NULL (only the shared expert's matrix is re-encoded, which is all the FP8
+ *   layer can use). ws (optional, may be NULL) receives the range flag in its status word.
  * Pass the results as moe_weights.w_down_f16 / ws_down_f16: moe_layer_forward,
  * moe_layer_forward_host and moe_grouped_swiglu then use them whenever they take the
  * tensor-core kernels (the down GEMM then runs on CTA pairs); the weight-streaming variant
@@ -330,8 +330,11 @@ moe_status moe_prepare_down_f16(const moe_shape* shape, const void* w_down, cons
  * scale per weight row:
  *   scale = amax_row / 448 (fp32 division; 0 for an all-zero row)
  *   code  = E4M3 round-to-nearest-even of (w / scale) (fp32 division), clamped to +-448
- * and the weight the layer uses is decode(code) * scale. Activations, h and the output
- * keep the precision of the bf16 layer.
+ * and the weight the layer uses is decode(code) * scale. Both GEMMs run E4M3 MMAs on the
+ * codes; the token operand goes in as exact E4M3 pieces with a power-of-two row scale: x as
+ * two (its bf16 value exactly, for elements within 2^9 of the row's largest), h as four
+ * (within 2^-16 of each element: the precision of the bf16 layer's hi + lo pair). fp32
+ * accumulation and output.
  *
  * moe_fp8_experts: q_gate_up uint8 [E][2I][H] (rows 0..I-1 gate, I..2I-1 up), s_gate_up
  *   fp32 [E][2I], q_down uint8 [E][H][I], s_down fp32 [E][H]. Device pointers, 16-byte
@@ -341,10 +344,9 @@ moe_status moe_prepare_down_f16(const moe_shape* shape, const void* w_down, cons
  *   Errors: MOE_ERR_INVALID_ARG (null or misaligned pointer), MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA.
  * moe_layer_forward_fp8: moe_layer_forward with the routed experts taken from `experts`
  *   (weights->w_gate_up and weights->w_down are not read and may be NULL). With
- *   weights->ws_down_f16 given (moe_prepare_down_f16), h is carried as one fp16 value and
- *   the codes are widened to fp16 for the down GEMM (one MMA per K step, deeper staging);
- *   without it, as the bf16 pair. Supported for
- *   decode-size batches, T*k < 16*E, with I and Is multiples of 128 and H of 256 on
+ *   weights->ws_down_f16 given (moe_prepare_down_f16 with no routed pair), the shared
+ *   expert's down GEMM takes h's shared rows as one fp16 value (11 significant bits)
+ *   instead of the pair. Any batch size, with I and Is multiples of 128 and H of 256 on
  *   sm_100; otherwise MOE_ERR_UNSUPPORTED. Same outputs, workspace and errors as
  *   moe_layer_forward.
  */

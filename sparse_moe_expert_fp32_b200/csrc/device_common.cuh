@@ -109,5 +109,46 @@ __device__ inline int block_exclusive_scan(int v, int* smem_warp, int* total) {
   return r;
 }
 
+// N block-wide exclusive scans at once (one value of each per thread, one set of barriers);
+// blockDim.x must be kScanThreads. smem_warp holds 33 * N ints.
+template <int N>
+__device__ inline void block_exclusive_scan_n(const int (&v)[N], int (&prefix)[N],
+                                              int (&total)[N], int* smem_warp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl[N];
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    incl[j] = v[j];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl[j], o);
+      if (lane >= o) incl[j] += n;
+    }
+    if (lane == 31) smem_warp[j * 33 + warp] = incl[j];
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const int s = smem_warp[j * 33 + lane];
+      int si = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, si, o);
+        if (lane >= o) si += n;
+      }
+      smem_warp[j * 33 + lane] = si - s;  // exclusive warp prefix
+      if (lane == 31) smem_warp[j * 33 + 32] = si;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    prefix[j] = smem_warp[j * 33 + warp] + incl[j] - v[j];
+    total[j] = smem_warp[j * 33 + 32];
+  }
+  __syncthreads();
+}
+
 
 }  // namespace moe

@@ -4,6 +4,7 @@
 // Dispatch R tokens -> Grouped expert GEMMs -> Weighted combine + gated shared expert").
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <unordered_map>
@@ -28,9 +29,11 @@ Layout layout(const moe_shape& s) {
     return at;
   };
   L.status = take(64 * sizeof(uint32_t));
-  // below 512 tokens the router keeps four partial sums per logit; the region is sized so
-  // that the workspace never shrinks as T grows (a workspace for T serves every T' <= T)
-  const size_t logit_rows = T < 512 ? 4 * T : (T > 2044 ? T : 2044);
+  // below 512 tokens the router keeps kRouterSplits partial sums per logit; the region is
+  // sized so that the workspace never shrinks as T grows (a workspace for T serves every
+  // T' <= T)
+  const size_t small_max = (size_t)kRouterSplits * 511;
+  const size_t logit_rows = T < 512 ? kRouterSplits * T : (T > small_max ? T : small_max);
   L.logits = take(logit_rows * E * sizeof(float));
   L.wr_split = take(E * 3 * H * sizeof(uint16_t));
   L.ids = take(R * sizeof(int32_t));
@@ -45,7 +48,8 @@ Layout layout(const moe_shape& s) {
   L.assign_row = take(R * sizeof(int32_t));
   L.plan = take(plan_ints(s.E) * sizeof(int32_t));
   L.sched = take(4 * sizeof(int32_t));
-  L.xs = take(R * H * sizeof(uint16_t));
+  // the FP8 layer reuses it for h's E4M3 pieces and their row scales once gate|up has run
+  L.xs = take(std::max(R * H * sizeof(uint16_t), fp8_h_pieces_bytes(s) + R * sizeof(float)));
   L.h_plane = (R + T) * (size_t)L.ldh;
   L.h = take(2 * L.h_plane * sizeof(uint16_t));
   L.total = o;
@@ -519,8 +523,7 @@ moe_status moe_layer_forward_fp8(const moe_shape* shape, const void* x, const mo
                           sorted_token, sorted_w, reinterpret_cast<int32_t*>(w + L.assign_row),
                           st));
   MOE_CUDA(launch_tc8_gate_up(s, L, w, xb, sorted_token, *weights, *experts, st));
-  MOE_CUDA(launch_tc8_down(s, L, w, sorted_token, sorted_w, sg, *weights, *experts, nullptr,
-                           nullptr, out, st));
+  MOE_CUDA(launch_tc8_down(s, L, w, sorted_token, sorted_w, sg, *weights, *experts, out, st));
   return MOE_OK;
 }
 

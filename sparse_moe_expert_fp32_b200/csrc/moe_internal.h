@@ -23,8 +23,8 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Byte offsets of the workspace regions (all 256-byte aligned).
 struct Layout {
   size_t status;        // uint32 [64]: [0] = error flags, [1..] = diagnostics
-  size_t logits;        // fp32 [4][T][E] partial router logits for T < 512, else [T][E]
-                        // (at least 2044 x E entries from T = 512 on: sizes grow with T)
+  size_t logits;        // fp32 [8][T][E] partial router logits for T < 512, else [T][E]
+                        // (at least 8 x 511 x E entries from T = 512 on: sizes grow with T)
   size_t wr_split;      // bf16 [E][3H]: router matrix as hi|mid|lo bf16 pieces (tensor-core router)
   size_t ids;           // int32 [T][k]
   size_t w;             // fp32 [T][k]
@@ -59,9 +59,11 @@ struct PlanView {
   int* tp1;       // [E+2] tile prefix of the tensor-core gate|up GEMM
   int* tp2;       // [E+2] tile prefix of the tensor-core down GEMM (bf16 h pair, 128 rows)
   int* tp3;       // [E+2] tile prefix of the down GEMM on fp16 operands (256 rows)
+  int* tp4;       // [E+2] tile prefix of the FP8 gate|up GEMM (64 rows at every batch size)
+  int* tp5;       // [E+2] tile prefix of the FP8 down GEMM (32 rows)
 };
 
-__host__ __device__ inline size_t plan_ints(int E) { return 1 + (size_t)(E + 1) + 4 * (size_t)(E + 2); }
+__host__ __device__ inline size_t plan_ints(int E) { return 1 + (size_t)(E + 1) + 6 * (size_t)(E + 2); }
 
 __host__ __device__ inline PlanView plan_view(void* base, int E) {
   int* p = static_cast<int*>(base);
@@ -72,6 +74,8 @@ __host__ __device__ inline PlanView plan_view(void* base, int E) {
   v.tp1 = v.row0 + (E + 2);
   v.tp2 = v.tp1 + (E + 2);
   v.tp3 = v.tp2 + (E + 2);
+  v.tp4 = v.tp3 + (E + 2);
+  v.tp5 = v.tp4 + (E + 2);
   return v;
 }
 
@@ -85,11 +89,25 @@ constexpr int kTcChunkDownF16 = 256;
 // fit; larger batches at kTcChunk. The plan builder and both gate|up kernels call this with
 // the same T, k, E.
 constexpr int kTcChunkSmall = 64;
+// Rows per tile of the FP8 kernels, whatever the batch size: gate|up 64 (the token operand
+// is two E4M3 pieces, MMA N = 2 x rows), down 32 (h is four pieces, MMA N = 4 x rows; both
+// accumulators of a tile then fit in one 256-column TMEM slot).
+constexpr int kTcChunkGateUp8 = 64;
+constexpr int kTcChunkDown8 = 32;
 __host__ __device__ inline int tc_gate_up_chunk(int T, int k, int E) {
   return (long long)T * k < 16LL * E ? kTcChunkSmall : kTcChunk;
 }
 __host__ __device__ inline int tc_nchunks(int n, int max_rows) {
   return (n + max_rows - 1) / max_rows;
+}
+
+// Hidden-dimension slices of the small-batch router's partial logits.
+constexpr int kRouterSplits = 8;
+
+// Bytes of the FP8 down GEMM's token operand: four E4M3 pieces of every routed row of h
+// (T*k rows of I codes), 256-byte aligned; the fp32 row scales follow.
+inline size_t fp8_h_pieces_bytes(const moe_shape& s) {
+  return align_up((size_t)4 * s.T * s.k * s.I, 256);
 }
 
 // ---------------------------------------------------------------- launch bookkeeping
@@ -105,8 +123,9 @@ struct LaunchScope {
 // ---------------------------------------------------------------- kernel launches
 // Every launcher enqueues on `st` and returns cudaGetLastError().
 
-// Router logits by the best kernel for the shape (uses the workspace). Small batches leave
-// router_slices(s) partial sums [slices][T][E] that launch_router_topk adds up.
+// Router logits by the best kernel for the shape (uses the workspace). Small batches
+// (T < 512) leave router_slices(s) = kRouterSplits partial sums [slices][T][E] that
+// launch_router_topk adds up in order.
 cudaError_t launch_router_logits(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                                  const float* wr, float* logits, cudaStream_t st);
 int router_slices(const moe_shape& s);

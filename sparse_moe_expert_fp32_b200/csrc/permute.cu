@@ -57,7 +57,7 @@ dispatch_mask_kernel(const int32_t* __restrict__ ids, int T, int E, int k,
 // Group sizes n_g (g < E routed, g == E shared = T) -> plan. Called by all threads of a
 // kScanThreads CTA; thread g handles group g (E + 1 <= 1025: thread 0 also takes E).
 __device__ void build_plan(const int* n_of, int E, int H, int I, int Is, int T, int k,
-                           PlanView pv, int* smem) {
+                           PlanView pv) {
   // thread g takes group g (g <= E); with E == 1024 the last thread also takes group E
   const int g = threadIdx.x;
   int n0 = 0, n1 = 0, has1 = 0;
@@ -65,45 +65,60 @@ __device__ void build_plan(const int* n_of, int E, int H, int I, int Is, int T, 
   if (g == kScanThreads - 1 && E == kScanThreads) { n1 = n_of[E]; has1 = 1; }
   const int a0 = (g <= E && g < kScanThreads && n0 > 0) ? 1 : 0;
   const int a1 = (has1 && n1 > 0) ? 1 : 0;
-  int tot;
-  const int pos = block_exclusive_scan(a0 + a1, smem, &tot);
-  if (a0) pv.active[pos] = g;
-  if (a1) pv.active[pos + a0] = E;
-  if (threadIdx.x == 0) *pv.n_active = tot;
 
   auto inter = [&](int grp) { return grp < E ? I : Is; };
   const int uc = tc_gate_up_chunk(T, k, E);
   const int c0 = tc_nchunks(n0, uc), c1 = tc_nchunks(n1, uc);
   const int d0 = tc_nchunks(n0, kTcChunkDown), d1 = tc_nchunks(n1, kTcChunkDown);
   const int f0 = tc_nchunks(n0, kTcChunkDownF16), f1 = tc_nchunks(n1, kTcChunkDownF16);
+  const int q0 = tc_nchunks(n0, kTcChunkGateUp8), q1 = tc_nchunks(n1, kTcChunkGateUp8);
+  const int e0 = tc_nchunks(n0, kTcChunkDown8), e1 = tc_nchunks(n1, kTcChunkDown8);
   const int t1a = (g <= E) ? c0 * (inter(g) / 128) : 0;
   const int t1b = has1 ? c1 * (Is / 128) : 0;
   const int t2a = (g <= E) ? d0 * (H / 256) : 0;
   const int t2b = has1 ? d1 * (H / 256) : 0;
   const int t3a = (g <= E) ? f0 * (H / 256) : 0;
   const int t3b = has1 ? f1 * (H / 256) : 0;
+  const int t4a = (g <= E) ? q0 * (inter(g) / 128) : 0;
+  const int t4b = has1 ? q1 * (Is / 128) : 0;
+  const int t5a = (g <= E) ? e0 * (H / 256) : 0;
+  const int t5b = has1 ? e1 * (H / 256) : 0;
   const int r0a = (g <= E) ? n0 : 0, r0b = has1 ? n1 : 0;
-  int tot1, tot2, tot3, totr;
-  const int p1 = block_exclusive_scan(t1a + t1b, smem, &tot1);
-  const int p2 = block_exclusive_scan(t2a + t2b, smem, &tot2);
-  const int p3 = block_exclusive_scan(t3a + t3b, smem, &tot3);
-  const int pr = block_exclusive_scan(r0a + r0b, smem, &totr);
+  // the active groups, the five tile prefixes and the row prefix in one pass
+  __shared__ int scan7[33 * 7];
+  const int vals[7] = {a0 + a1,   t1a + t1b, t2a + t2b, t3a + t3b,
+                       t4a + t4b, t5a + t5b, r0a + r0b};
+  int pre[7], tot[7];
+  block_exclusive_scan_n<7>(vals, pre, tot, scan7);
+  const int pos = pre[0];
+  if (a0) pv.active[pos] = g;
+  if (a1) pv.active[pos + a0] = E;
+  if (threadIdx.x == 0) *pv.n_active = tot[0];
+  const int p1 = pre[1], p2 = pre[2], p3 = pre[3], p4 = pre[4], p5 = pre[5], pr = pre[6];
+  const int tot1 = tot[1], tot2 = tot[2], tot3 = tot[3], tot4 = tot[4], tot5 = tot[5],
+            totr = tot[6];
   if (g <= E) {
     pv.tp1[g] = p1;
     pv.tp2[g] = p2;
     pv.tp3[g] = p3;
+    pv.tp4[g] = p4;
+    pv.tp5[g] = p5;
     pv.row0[g] = pr;
   }
   if (has1) {
     pv.tp1[E] = p1 + t1a;
     pv.tp2[E] = p2 + t2a;
     pv.tp3[E] = p3 + t3a;
+    pv.tp4[E] = p4 + t4a;
+    pv.tp5[E] = p5 + t5a;
     pv.row0[E] = pr + r0a;
   }
   if (threadIdx.x == 0) {
     pv.tp1[E + 1] = tot1;
     pv.tp2[E + 1] = tot2;
     pv.tp3[E + 1] = tot3;
+    pv.tp4[E + 1] = tot4;
+    pv.tp5[E + 1] = tot5;
     pv.row0[E + 1] = totr;
   }
 }
@@ -135,7 +150,7 @@ dispatch_scan_kernel(const int32_t* blk_count, int nblk, int T, int E, int k, in
     n_of[E] = T;
   }
   __syncthreads();
-  build_plan(n_of, E, H, I, Is, T, k, plan_view(plan_base, E), smem);
+  build_plan(n_of, E, H, I, Is, T, k, plan_view(plan_base, E));
 }
 
 __global__ void __launch_bounds__(kPermBlock)
@@ -208,7 +223,7 @@ dispatch_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__
     n_of[E] = T;
   }
   __syncthreads();
-  build_plan(n_of, E, H, I, Is, T, k, plan_view(plan_base, E), smem);
+  build_plan(n_of, E, H, I, Is, T, k, plan_view(plan_base, E));
   if (i < T) {
     const int word = i >> 5;
     const uint32_t below = (1u << (i & 31)) - 1u;
@@ -232,7 +247,6 @@ __global__ void __launch_bounds__(kScanThreads)
 plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int T, int E, int k, int H, int I,
                          int Is, int shared_rows, int* __restrict__ plan_base,
                          uint32_t* __restrict__ status) {
-  __shared__ int smem[33];
   __shared__ int n_of[kMaxE + 1];
   __shared__ int bad;
   if (threadIdx.x == 0) bad = (offsets[0] != 0 || offsets[E] > T * k) ? 1 : 0;
@@ -249,7 +263,7 @@ plan_from_offsets_kernel(const int32_t* __restrict__ offsets, int T, int E, int 
     if (threadIdx.x == 0) set_flag(status, kFlagBounds);
   }
   __syncthreads();
-  build_plan(n_of, E, H, I, Is, T, k, plan_view(plan_base, E), smem);
+  build_plan(n_of, E, H, I, Is, T, k, plan_view(plan_base, E));
 }
 
 }  // namespace

@@ -4,7 +4,7 @@
 // output gate).
 //
 //   router_logits_small_kernel  : logits = x . Wr^T on CUDA cores for small batches, as
-//                                 four partial sums over hidden-dimension slices; larger
+//                                 eight partial sums over hidden-dimension slices; larger
 //                                 batches use the tensor-core router in tc_gemm.cu.
 //   router_topk_kernel          : two warps per token: one takes the top-k with
 //                                 lowest-index ties, the renormalised softmax weights and
@@ -22,38 +22,44 @@
 namespace moe {
 namespace {
 
-// Small batches (T < 512): partial logits over kSplits slices of the hidden dimension,
-// part[s][t][e] = sum_{h in slice s} x[t][h] * wr[e][h], fp32 FMAs in h order. A CTA
-// computes 16 experts x 64 tokens of one slice: x and wr chunks of 128 hidden positions are
-// staged in shared memory (x transposed so that a warp's 32 tokens read consecutive words),
-// double-buffered -- the next chunk's global loads are in flight while the current one is
-// multiplied -- and each thread accumulates 4 experts x 1 token. The top-k kernel adds the
-// slices in order s = 0..3, so the logits are the same on every run. Grid
-// (ceil(E/16), kSplits, ceil(T/64)) fills the GPU at decode sizes (128 CTAs at E = 512,
-// T = 64) and reads wr once.
-constexpr int kSplits = 4;
-constexpr int kSmallTok = 64;
-constexpr int kSmallExp = 16;
-constexpr int kSmallKc = 128;
+// Small batches (T < 512): partial logits over kRouterSplits slices of the hidden
+// dimension, part[s][t][e] = sum_{h in slice s} x[t][h] * wr[e][h], fp32 FMAs in h order. A
+// CTA computes 32 tokens x 64 experts of one slice: x and wr chunks of 320 hidden positions
+// (the whole slice at hidden 2560; 120 KB) are staged in shared memory (both transposed: x
+// as [h][token], wr as [h][expert]). All of a chunk's global loads are issued at once, into
+// registers, so their latency is paid once per chunk; the next chunk's loads are in flight
+// while the current one is multiplied. Each thread accumulates 2 tokens x 4 experts: an
+// 8-byte and a 16-byte
+// shared-memory load (one wavefront each per warp) feed 8 FMAs, so the FMA pipe, not shared
+// memory, sets the pace. The top-k kernel adds the slices in order s = 0 .. kRouterSplits-1,
+// so the logits are the same on every run. Grid (ceil(E/64), kRouterSplits, ceil(T/32)):
+// 128 CTAs at E = 512, T = 64; wr is read once per token block.
+constexpr int kSplits = kRouterSplits;
+constexpr int kSmallTok = 32;
+constexpr int kSmallExp = 64;
+constexpr int kSmallKc = 320;
 constexpr int kSmallThreads = 256;
 constexpr int kSmallXLoads = kSmallTok * (kSmallKc / 8) / kSmallThreads;  // uint4 per thread
 constexpr int kSmallWLoads = kSmallExp * (kSmallKc / 4) / kSmallThreads;  // float4 per thread
-constexpr size_t kSmallSmem =
-    2 * (size_t)kSmallKc * kSmallTok * sizeof(float) + 2 * (size_t)kSmallKc * kSmallExp * sizeof(float);
+constexpr size_t kSmallSmem = (size_t)kSmallKc * (kSmallTok + kSmallExp) * sizeof(float);
+static_assert(kSmallXLoads * kSmallThreads * 8 == kSmallTok * kSmallKc, "x chunk split");
+static_assert(kSplits % 4 == 0, "the top-k kernel adds the slices two or four at a time");
+static_assert(kSmallWLoads * kSmallThreads * 4 == kSmallExp * kSmallKc, "wr chunk split");
 
 __global__ void __launch_bounds__(kSmallThreads)
 router_logits_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
                            float* __restrict__ part, int T, int H, int E, int nslices) {
   extern __shared__ float4 dsm[];
-  float* xs_all = reinterpret_cast<float*>(dsm);                            // [2][Kc][Tok]
-  float* ws_all = xs_all + 2 * kSmallKc * kSmallTok;                       // [2][Kc][Exp]
+  float* xs_all = reinterpret_cast<float*>(dsm);  // [Kc][Tok]
+  float* ws_all = xs_all + kSmallKc * kSmallTok;  // [Kc][Exp]
   const int e0 = blockIdx.x * kSmallExp;
   const int t0 = blockIdx.z * kSmallTok;
-  const int slice = H / nslices;  // a multiple of 16 (H is a multiple of 64)
+  const int slice = H / nslices;  // a multiple of 8 (H is a multiple of 64)
   const int kbeg = blockIdx.y * slice, kend = kbeg + slice;
   const int tid = threadIdx.x;
-  const int tok = tid & (kSmallTok - 1), eg = tid >> 6;  // 4 expert groups of 4
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int tg = tid & 15;  // tokens 2 tg, 2 tg + 1
+  const int eg = tid >> 4;  // experts 4 eg .. 4 eg + 3
+  float acc[2][4] = {};
   uint4 xr[kSmallXLoads];
   float4 wv[kSmallWLoads];
 
@@ -76,10 +82,10 @@ router_logits_small_kernel(const uint16_t* __restrict__ x, const float* __restri
         wv[q] = __ldg(reinterpret_cast<const float4*>(wr + (size_t)(e0 + e) * H + k0) + c);
     }
   };
-  // registers -> shared-memory buffer b
-  auto store = [&](int b) {
-    float* xs = xs_all + b * kSmallKc * kSmallTok;
-    float* ws = ws_all + b * kSmallKc * kSmallExp;
+  // registers -> shared memory
+  auto store = [&]() {
+    float* xs = xs_all;
+    float* ws = ws_all;
 #pragma unroll
     for (int q = 0; q < kSmallXLoads; ++q) {
       const int i = tid + q * kSmallThreads;
@@ -101,34 +107,47 @@ router_logits_small_kernel(const uint16_t* __restrict__ x, const float* __restri
   };
 
   load(kbeg);
-  store(0);
+  store();
   __syncthreads();
-  int b = 0;
-  for (int k0 = kbeg; k0 < kend; k0 += kSmallKc, b ^= 1) {
+  for (int k0 = kbeg; k0 < kend; k0 += kSmallKc) {
     const bool more = k0 + kSmallKc < kend;
     if (more) load(k0 + kSmallKc);
-    const int kn = min(kSmallKc, kend - k0);
-    const float* xs = xs_all + b * kSmallKc * kSmallTok;
-    const float4* ws = reinterpret_cast<const float4*>(ws_all + b * kSmallKc * kSmallExp);
-    for (int kk = 0; kk < kn; ++kk) {
-      const float xv = xs[kk * kSmallTok + tok];
-      const float4 w = ws[kk * (kSmallExp / 4) + eg];
-      acc[0] = fmaf(xv, w.x, acc[0]);
-      acc[1] = fmaf(xv, w.y, acc[1]);
-      acc[2] = fmaf(xv, w.z, acc[2]);
-      acc[3] = fmaf(xv, w.w, acc[3]);
+    const int kn = min(kSmallKc, kend - k0);  // a multiple of 8
+    const float2* xs = reinterpret_cast<const float2*>(xs_all) + tg;
+    const float4* ws = reinterpret_cast<const float4*>(ws_all) + eg;
+    for (int kk = 0; kk < kn; kk += 8) {
+      float2 x2[8];
+      float4 wv4[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        x2[u] = xs[(kk + u) * (kSmallTok / 2)];
+        wv4[u] = ws[(kk + u) * (kSmallExp / 4)];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {  // h order within each accumulator
+        const float xa[2] = {x2[u].x, x2[u].y};
+        const float wa[4] = {wv4[u].x, wv4[u].y, wv4[u].z, wv4[u].w};
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], wa[j], acc[i][j]);
+      }
     }
-    // the other buffer was last read before the barrier that ended the previous chunk
-    if (more) store(b ^ 1);
-    __syncthreads();
+    if (more) {
+      __syncthreads();  // every thread is done reading this chunk
+      store();
+      __syncthreads();
+    }
   }
-  const int t = t0 + tok;
-  if (t < T) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int t = t0 + 2 * tg + i;
+    if (t >= T) break;
     float* row = part + ((size_t)blockIdx.y * T + t) * E;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int e = e0 + eg * 4 + j;
-      if (e < E) row[e] = acc[j];
+      const int e = e0 + 4 * eg + j;
+      if (e < E) row[e] = acc[i][j];
     }
   }
 }
@@ -250,26 +269,35 @@ router_topk_kernel(const float* __restrict__ logits, const float* __restrict__ b
     return;
   }
 
-  float part[NS][VPL];
+  // slices added in order, a group of SG slices in flight at a time (SG * VPL loads)
+  constexpr int SG = NS < 4 ? NS : (VPL >= 32 ? 2 : 4);
+  float v[VPL];
 #pragma unroll
-  for (int sl = 0; sl < NS; ++sl)
+  for (int g = 0; g < NS; g += SG) {
+    float part[SG][VPL];
+#pragma unroll
+    for (int sl = 0; sl < SG; ++sl)
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int e = lane + 32 * i;
+        part[sl][i] = e < E ? logits[((size_t)(g + sl) * T + t) * E + e] : 0.f;
+      }
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      const int e = lane + 32 * i;
-      part[sl][i] = e < E ? logits[((size_t)sl * T + t) * E + e] : 0.f;
+      float l = g == 0 ? part[0][i] : v[i] + part[0][i];
+#pragma unroll
+      for (int sl = 1; sl < SG; ++sl) l += part[sl][i];
+      v[i] = l;
     }
-  float v[VPL];
+  }
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
-    float l = -FLT_MAX;
     if (e < E) {
-      l = part[0][i];
-#pragma unroll
-      for (int sl = 1; sl < NS; ++sl) l += part[sl][i];
-      if (bias) l += bias[e];
+      if (bias) v[i] += bias[e];
+    } else {
+      v[i] = -FLT_MAX;
     }
-    v[i] = l;
   }
 
   int my_id;

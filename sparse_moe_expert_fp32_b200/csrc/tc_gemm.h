@@ -43,15 +43,16 @@ cudaError_t launch_tc2_down_f16(const moe_shape& s, const Layout& L, char* ws,
                                 float* y_shared, float* out, cudaStream_t st);
 
 // The same grouped GEMMs with the routed experts' weights in FP8 (E4M3 codes, one fp32 scale
-// per weight row; the shared expert stays bf16): one CTA per tile, codes widened to bf16 in
-// shared memory. Decode-size batches only (T*k < 16*E), on tensor-core shapes.
+// per weight row; the shared expert stays bf16): one CTA per tile, E4M3 MMAs on the codes
+// against E4M3 pieces of the token operand (two for x, four for h; the down launcher splits
+// h first). Any batch size on tensor-core shapes; the down GEMM always combines into `out`.
 bool tc8_supported(const moe_shape& s);
 cudaError_t launch_tc8_gate_up(const moe_shape& s, const Layout& L, char* ws, const uint16_t* x,
                                const int32_t* sorted_token, const moe_weights& w,
                                const moe_fp8_experts& q, cudaStream_t st);
 cudaError_t launch_tc8_down(const moe_shape& s, const Layout& L, char* ws,
                             const int32_t* sorted_token, const float* sorted_w, const float* sgate,
-                            const moe_weights& w, const moe_fp8_experts& q, float* y,
-                            float* y_shared, float* out, cudaStream_t st);
+                            const moe_weights& w, const moe_fp8_experts& q, float* out,
+                            cudaStream_t st);
 
 }  // namespace moe

@@ -9,9 +9,12 @@ include/moe.h and in the oracle.
   sides, so its codes and scales must equal the oracle's bit for bit.
 * The layer (moe_layer_forward_fp8) must match the fp64 oracle evaluated on the
   dequantised FP8 bank within the layer tolerance (the FP8 rounding is part of the model,
-  not of the error): decode-size batches, several tile geometries, zero rows, rows whose
-  codes are nearly all E4M3 subnormals, and the Flash-Next decode layer at full size in the
-  configuration `bench.py --fp8` times.
+  not of the error): decode- and prefill-size batches, several tile geometries, zero rows,
+  rows whose codes are nearly all E4M3 subnormals, and the Flash-Next decode and prefill
+  layers at full size and the 2.4T-shaped prefill geometry (sampled tokens), in the
+  configurations `bench.py --fp8` times. Each case runs with the shared expert's down
+  matrix in bf16 (h's shared rows as the pair) and as fp16(W 2^8) (h's shared rows as
+  fp16(h 2^-8)); the routed rows of h always go in as four E4M3 pieces.
 """
 import numpy as np
 import pytest
@@ -28,8 +31,10 @@ from parity_util import assert_layer_close, id_sets_match  # noqa: E402
 
 TINY = synth.CONFIGS["tiny"]
 CASES = {
-    # T*k < 16*E in every case: the FP8 path serves decode-size batches
+    # decode-size (T*k < 16*E) and prefill-size batches
     "tiny_T48": dict(T=48),
+    "prefill_T600": dict(T=600),
+    "prefill_T257_k1": dict(T=257, k=1),
     "T1": dict(T=1),
     "T3_ragged": dict(T=3),
     "E1": dict(T=8, E=1, k=1),
@@ -53,8 +58,7 @@ def _quantize(cfg, dev):
 
 
 def _forward_fp8(cfg, dev, q, f16=False):
-    """The FP8 layer; with f16, on the fp16 down operands (the shared expert's matrix
-    re-encoded, h as one fp16 value, codes widened to fp16)."""
+    """The FP8 layer; with f16, the shared expert's down matrix as fp16(W 2^8)."""
     s = moe.shape_of(cfg)
     ws = moe.alloc_workspace(s)
     out = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
@@ -115,7 +119,6 @@ def test_quantize_bitexact_flash_decode_experts():
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_fp8_layer_small(case, f16):
     cfg = TINY.replace(name=case, **CASES[case])
-    assert cfg.T * cfg.k < 16 * cfg.E
     dev = synth.device_inputs(cfg, seed=4)
     host = synth.host_inputs(cfg, seed=4)
     q = _quantize(cfg, dev)
@@ -128,8 +131,9 @@ def test_fp8_layer_small(case, f16):
 @pytest.mark.gpu
 @pytest.mark.parametrize("f16", [False, True])
 def test_fp8_layer_hot_expert_several_tiles(f16):
-    """Every token on expert 7: 200 routed rows in one group (four 64-row gate|up tiles, two
-    112-row down tiles that take both TMEM slots) and 200 shared rows."""
+    """Every token on expert 7: 200 routed rows in one group (four 64-row gate|up tiles, of
+    which the last holds 8 rows; seven 32-row down tiles, the last with 8 rows in a 16-row
+    MMA) and 200 shared rows."""
     cfg = TINY.replace(name="hot_decode", T=200, E=256, k=4)
     assert cfg.T * cfg.k < 16 * cfg.E
     dev = synth.device_inputs(cfg, seed=8)
@@ -192,16 +196,31 @@ def test_fp8_layer_flash_decode_sampled(f16):
     print("flash_decode fp8", stats, "near-ties", ties)
 
 
+def _fp8_full_size(name, n_rows, f16):
+    cfg = synth.CONFIGS[name]
+    dev = synth.device_inputs(cfg, seed=0)
+    q = _quantize(cfg, dev)
+    out, ids = _forward_fp8(cfg, dev, q, f16)
+    del dev, q
+    torch.cuda.empty_cache()
+    host = synth.host_inputs(cfg, seed=0)
+    fp8 = oracle.Fp8Experts(host.gate_up, host.down)
+    rng = np.random.default_rng(78)
+    rows = sorted(set([0, cfg.T - 1] + rng.choice(cfg.T, n_rows, replace=False).tolist()))
+    stats, ties = _check(cfg, host, fp8, out, ids, rows)
+    print(name, "fp8", f16, stats, "near-ties", ties)
+
+
 @pytest.mark.gpu
-def test_fp8_rejects_prefill_size_batches():
-    cfg = synth.CONFIGS["flash_prefill"]  # T*k >= 16*E
-    s = moe.shape_of(cfg)
-    w = moe.moe_weights(16, 0, 0, 0, 64, 80, 96)
-    q = moe.moe_fp8_experts(4096, 8192, 12288, 16384)
-    ws = moe.alloc_workspace(moe.shape_of(cfg, T=1))  # any aligned pointer: nothing launches
-    before = moe.moe_launch_count()
-    st = moe.lib().moe_layer_forward_fp8(moe.ctypes.byref(s), 16, moe.ctypes.byref(w),
-                                         moe.ctypes.byref(q), 16, None, None, None, ws.data_ptr(),
-                                         moe.moe_workspace_bytes(s), None)
-    assert st == moe.MOE_ERR_UNSUPPORTED
-    assert moe.moe_launch_count() == before
+@pytest.mark.parametrize("f16", [False, True])
+def test_fp8_layer_flash_prefill_sampled(f16):
+    """The Flash-Next prefill layer at full size (T=8192, E=512, k=10): 160 rows per expert,
+    three 64-row gate|up tiles and five 32-row down tiles per group."""
+    _fp8_full_size("flash_prefill", 14, f16)
+
+
+@pytest.mark.gpu
+def test_fp8_layer_t24_prefill_e16_sampled():
+    """The 2.4T-shaped prefill geometry (H=8192, I=2048, 160 rows per expert) on the
+    16-expert profiling case."""
+    _fp8_full_size("t24_prefill_e16", 24, True)
