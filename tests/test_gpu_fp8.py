@@ -39,6 +39,8 @@ CASES = {
     "T3_ragged": dict(T=3),
     "E1": dict(T=8, E=1, k=1),
     "zero_rows": dict(T=48, zero_rows_pct=50),
+    "E_eq_k": dict(T=24, E=4, k=4),
+    "max_E_k": dict(T=40, E=1024, k=32),
     "shared_narrower": dict(T=40, I=256, Is=128),
 }
 
