@@ -274,6 +274,42 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const void* tmap, ui
       : "memory");
 }
 
+// L2 cache policy for data read once (a streamed weight tile): its lines are the first to
+// be evicted, so that lines in reuse (accumulated outputs, shared operands) stay.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// L2 cache policy for data in reuse (a row accumulated by many atomic adds): its lines are
+// the last to be evicted.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Four fp32 atomic adds at a 16-byte-aligned address (a reduction, no return value), with
+// an L2 cache policy for the line.
+__device__ __forceinline__ void red_add_v4_f32_hint(float* addr, float4 v, uint64_t policy) {
+  asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(addr),
+               "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "l"(policy)
+               : "memory");
+}
+
+// tma_load_3d_pair with an L2 cache policy for the loaded lines.
+__device__ __forceinline__ void tma_load_3d_pair_hint(void* dst, const void* tmap,
+                                                      uint32_t bar_cluster_addr, int c0, int c1,
+                                                      int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2),
+      "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_5d_pair(void* dst, const void* tmap, uint32_t bar_cluster_addr,
                                                  int c0, int c1, int c2, int c3, int c4) {
   asm volatile(

@@ -219,6 +219,7 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     // full barrier with both CTAs' bytes); then lane 0 issues the weight box and lane 1 the
     // box of this CTA's token rows, each covering all KSUB K blocks of the stage.
     const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(&S.full[0]), 0);
+    const uint64_t evict_first = ptx::l2_policy_evict_first();
     int it = 0;
     bool aborted = false;
     for (int tile = pair; tile < total && !aborted; tile += npairs) {
@@ -244,8 +245,10 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         if (lane == 0) {
           if (MODE == kPairGateUp)  // [K block][gate, up][64 channels][64 K]
             ptx::tma_load_5d_pair(st, a_map, bar, 0, G.a_row0, 0, ks * KSUB, G.a_e);
-          else  // [K block][128 rows][64 K]
+          else if (G.shared)  // [K block][128 rows][64 K]; re-read by every token chunk
             ptx::tma_load_3d_pair(st, a_map, bar, 0, G.a_row0, ks * KSUB);
+          else  // routed weights are read once: evicted first, so out rows and h stay in L2
+            ptx::tma_load_3d_pair_hint(st, a_map, bar, 0, G.a_row0, ks * KSUB, evict_first);
         } else if (lane == 1) {  // [K block][nbb token rows][64 K]
           ptx::tma_load_3d_pair(st + kABytes, b_map, bar, 0, G.b_row, ks * KSUB);
         }
@@ -324,6 +327,9 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     const int half = (warp - 2) >> 2;  // which 32-column chunks this warp drains
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t tmem_empty0 = ptx::mapa_shared(ptx::smem_u32(&S.tmem_empty[0]), 0);
+    // out rows take k + 1 atomic adds each, from experts far apart in the tile order: keep
+    // their lines in L2 (evicted last) rather than fetch them from DRAM for every add
+    const uint64_t keep = ptx::l2_policy_evict_last();
     // gate|up: warps q = 0, 1 hold gate and q = 2, 3 up of the same 32 channels
     const int xp = half * 2 + (q & 1);  // warp pair index, 0..3
     // named barriers of the pair: its per-tile decision, "buffer free", "buffer full"
@@ -433,8 +439,8 @@ tc2_grouped_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
               if (col < tl.nvalid) {
                 const int p = tl.p0 + col;
                 if (args.out) {
-                  atomicAdd(reinterpret_cast<float4*>(args.out + (size_t)t * H + mrow),
-                            make_float4(w * v.x, w * v.y, w * v.z, w * v.w));
+                  ptx::red_add_v4_f32_hint(args.out + (size_t)t * H + mrow,
+                                           make_float4(w * v.x, w * v.y, w * v.z, w * v.w), keep);
                 } else {
                   float* row =
                       p < R ? args.y + (size_t)p * H : args.y_shared + (size_t)(p - R) * H;
