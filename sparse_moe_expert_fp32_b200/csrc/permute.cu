@@ -191,12 +191,25 @@ dispatch_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__
   __shared__ int smem[33];
   __shared__ int n_of[kMaxE + 1];
   __shared__ int base[kMaxE];
+  const int i = threadIdx.x;
+  // token i's first kPre expert ids and routing weights, loaded before anything waits on
+  // them (one round trip instead of one per assignment); later ones, if k > kPre, in the loops
+  constexpr int kPre = 12;
+  int my_ids[kPre];
+  float my_w[kPre];
+#pragma unroll
+  for (int j = 0; j < kPre; ++j) {
+    const bool have = i < T && j < k;
+    my_ids[j] = have ? ids[(size_t)i * k + j] : -1;
+    my_w[j] = (have && topk_w) ? topk_w[(size_t)i * k + j] : 0.f;
+  }
   for (int q = threadIdx.x; q < E * 8; q += blockDim.x) mask[q] = 0;
   __syncthreads();
-  const int i = threadIdx.x;
   if (i < T) {
-    for (int j = 0; j < k; ++j) {
-      const int e = ids[(size_t)i * k + j];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j >= k) break;
+      const int e = j < kPre ? my_ids[j] : ids[(size_t)i * k + j];
       if (e < 0 || e >= E) {
         set_flag(status, kFlagBounds);
         continue;
@@ -227,15 +240,17 @@ dispatch_small_kernel(const int32_t* __restrict__ ids, const float* __restrict__
   if (i < T) {
     const int word = i >> 5;
     const uint32_t below = (1u << (i & 31)) - 1u;
-    for (int j = 0; j < k; ++j) {
-      const int ee = ids[(size_t)i * k + j];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j >= k) break;
+      const int ee = j < kPre ? my_ids[j] : ids[(size_t)i * k + j];
       if (ee < 0 || ee >= E) continue;
       const uint32_t* m = mask + ee * 8;
       int rank = __popc(m[word] & below);
       for (int w = 0; w < word; ++w) rank += __popc(m[w]);
       const int p = base[ee] + rank;
       sorted_token[p] = i;
-      if (sorted_w) sorted_w[p] = topk_w[(size_t)i * k + j];
+      if (sorted_w) sorted_w[p] = j < kPre ? my_w[j] : topk_w[(size_t)i * k + j];
       assign_row[(size_t)i * k + j] = p;
     }
   }
