@@ -87,3 +87,30 @@ def test_four_piece_h_rows_bound():
     # the epilogue's fold ((p4/16 + p3)/16 + p2)/16 + p1 in fp32 is the same sum
     near = np.abs(v) >= 2.0 ** -6
     assert near.mean() > 0.9
+
+
+def test_four_piece_h_rows_edge_scales():
+    """Rows the pre-pass meets at the edges: an all-zero row (the kernel takes k = 0 there,
+    every piece is zero); a row whose largest magnitude is 2^-125 (k clamped at 120, so v
+    stays below 128 and the pieces carry it within the bound); a row of magnitude 2^100
+    (k = -93)."""
+    rows = np.zeros((3, 256), np.float64)
+    rows[1] = np.linspace(-1.0, 1.0, 256) * 2.0 ** -125
+    rows[2] = np.linspace(-1.0, 1.0, 256) * 2.0 ** 100
+    hi = _bf16_rn(rows)
+    lo = _bf16_rn(rows.astype(np.float32) - hi)
+    h = hi.astype(np.float32) + lo
+    k = _row_scale(h)
+    assert k[1] == 120 and k[2] == 7 - 100
+    k = np.where(np.abs(h).max(axis=1) > 0, k, 0)  # the kernel's choice for an all-zero row
+    v = (h.astype(np.float64) * np.exp2(k)[:, None]).astype(np.float32)
+    assert np.isfinite(v).all() and (np.abs(v) < 256).all()
+    r = v.copy()
+    total = np.zeros(v.shape, np.float64)
+    for j in range(4):
+        p = _e4m3(r)
+        total += p.astype(np.float64) * 16.0 ** -j
+        r = ((r - p).astype(np.float32) * 16).astype(np.float32)
+    assert not total[0].any()
+    err = np.abs(total - v)
+    assert (err <= np.maximum(np.abs(v).astype(np.float64) * 2.0 ** -16, 2.0 ** -22)).all()
