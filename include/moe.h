@@ -51,7 +51,8 @@ typedef enum moe_status {
   MOE_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed          */
   MOE_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device-side wait gave up            */
   MOE_ERR_DEVICE_BOUNDS = 6,       /* a kernel met an expert id outside [0, E)      */
-  MOE_ERR_DEVICE_RANGE = 7         /* a value saturated to fit fp16 (down operands)  */
+  MOE_ERR_DEVICE_RANGE = 7         /* a value saturated to fit fp16 (down operands),
+                                      or h held inf/NaN (FP8 layer)                 */
 } moe_status;
 
 /* Layer shape. T tokens, hidden size H, E routed experts, k experts per token,
@@ -373,8 +374,8 @@ moe_status moe_layer_forward_fp8(const moe_shape* shape, const void* x,
 moe_status moe_set_variant(moe_variant variant);
 moe_status moe_workspace_set_variant(void* ws, size_t ws_bytes, moe_variant variant);
 
-/* Synchronise `stream`, read the workspace status word (MOE_OK, MOE_ERR_DEVICE_BOUNDS
- * or MOE_ERR_DEVICE_TIMEOUT), and clear it. `detail` (HOST, may be NULL) receives
+/* Synchronise `stream`, read the workspace status word (MOE_OK, MOE_ERR_DEVICE_BOUNDS,
+ * MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_RANGE), and clear it. `detail` (HOST, may be NULL) receives
  * the raw flag bits. */
 moe_status moe_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* detail);
 
