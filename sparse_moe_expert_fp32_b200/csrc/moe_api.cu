@@ -656,7 +656,8 @@ const char* moe_status_string(moe_status status) {
     case MOE_ERR_CUDA: return "CUDA runtime or launch error";
     case MOE_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
     case MOE_ERR_DEVICE_BOUNDS: return "expert id out of range";
-    case MOE_ERR_DEVICE_RANGE: return "a value saturated to fit fp16 (down operands) or h held inf/NaN";
+    case MOE_ERR_DEVICE_RANGE:
+      return "a value saturated to fit fp16 (down operands) or h held inf/NaN";
   }
   return "unknown status";
 }
