@@ -251,17 +251,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// 2-D tiled load into this CTA's shared memory whose completed bytes are counted on the
-// mbarrier at `bar_cluster_addr` (the leader CTA's), as the pair MMA requires. No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* tmap,
-                                                 uint32_t bar_cluster_addr, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster_addr), "r"(c0), "r"(c1)
-      : "memory");
-}
-
 // The same for 3-D and 5-D boxes: one instruction brings a whole stage's operand (several
 // 64-element K blocks, and for gate|up the gate and the up rows), where 2-D boxes need one
 // instruction per block. Coordinates innermost first.
