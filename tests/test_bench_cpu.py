@@ -31,7 +31,7 @@ def test_decode_down_bytes_by_hand():
 
 def test_prefill_flops_match_the_layer_count():
     # 6*H*I per routed assignment plus 6*H*Is per token for the shared expert, split 2:1
-    # between gate|up and down (the survey's 805.3 G + 80.5 G for the Flash-Next prefill)
+    # between gate|up and down (805.3 G + 80.5 G for the Flash-Next prefill, counted by hand)
     cfg = synth.CONFIGS["flash_prefill"]
     total = bench.kernel_flops("gate_up", cfg) + bench.kernel_flops("down", cfg)
     assert total == 6 * (cfg.R * cfg.H * cfg.I + cfg.T * cfg.H * cfg.Is)
@@ -84,7 +84,7 @@ def test_reference_arm_times_the_fp8_oracle():
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
 
 
-def test_layer_totals_match_the_survey_counts():
+def test_layer_totals_match_hand_counts():
     # 2.4T-shaped prefill, every expert active: routed 8.246 TFLOP + shared 0.825 TFLOP +
     # router 68.7 GFLOP; 51.54 GB of routed weights + shared expert + router matrix + x + out
     # (fp32) = 52.06 GB
